@@ -1,0 +1,249 @@
+/*
+ * stepq.h -- C ABI of the B200 (sm_100a) quantised gated Delta-rule decode step.
+ *
+ * The method is STEPQuant ("STEPQuant: When and Where Errors Matter in
+ * Delta-Rule Recurrent State Quantization").  Each request keeps, per head, a
+ * recurrent state S (d_k key rows x d_v value columns) stored packed: low-bit
+ * integer codes times a row factor and a column factor, S = codes (.) (r c^T),
+ * with FP16 "pivot" units kept raw (hyper.ai summary, "Method": symmetric
+ * uniform quantisation, FP16 sparse pivots, key-row-aware dual-axis fitting;
+ * rcap.io post, decode-step pseudocode).  One decode step of one (request,
+ * head) reads the packed state, reconstructs it, applies the gated Delta
+ * update, emits the readout y = X^T q before requantising, refits the row and
+ * column scales and writes the state back packed (rcap.io post, decode-step
+ * pseudocode; hyper.ai summary, "Method", last paragraph: a fused kernel for
+ * reconstruction + Delta update + readout, and the dual-axis fit + pack
+ * write-back on a separate CUDA stream).
+ *
+ * Conventions for every entry point:
+ *   - returns STEPQ_OK (0) or an error code below; nothing else crosses the
+ *     ABI (no exceptions).  stepq_last_error() gives a message for the last
+ *     failing call on the calling thread.
+ *   - "device" pointers are CUDA device (or managed) memory of the current
+ *     device; "host" pointers are ordinary host memory.  All arrays are dense,
+ *     C order, and must be aligned to 16 bytes.
+ *   - `stream` arguments are cudaStream_t values passed as void* (NULL = the
+ *     legacy default stream).  Device work is enqueued asynchronously; a
+ *     call returns once its kernels are launched.
+ *   - argument errors are reported as STEPQ_ERR_INVALID before anything is
+ *     launched; CUDA launch errors as STEPQ_ERR_CUDA.  Errors found by the
+ *     kernels themselves (a slot index outside the pool, a non-finite updated
+ *     state, a device wait that gave up) are recorded in the pool's device
+ *     status word, read with stepq_get_status().
+ *   - the library allocates device memory only in stepq_plan_create (its
+ *     tables) and stepq_pool_alloc (a status word); every buffer passed in
+ *     stays owned by the caller.
+ */
+#ifndef STEPQ_H
+#define STEPQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define STEPQ_API __attribute__((visibility("default")))
+#else
+#define STEPQ_API
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define STEPQ_OK 0
+#define STEPQ_ERR_INVALID 1     /* bad argument, caught on the host          */
+#define STEPQ_ERR_CUDA 2        /* a CUDA runtime call or launch failed      */
+#define STEPQ_ERR_UNSUPPORTED 3 /* valid but not built for (e.g. d_k != d_v) */
+
+/* ---- bits of the device status word (stepq_get_status) ----------------- */
+#define STEPQ_DEV_BAD_SLOT 1u   /* a slot index was outside [0, num_slots); that head was skipped */
+#define STEPQ_DEV_NONFINITE 2u  /* an updated state row held NaN/Inf; it was stored as zeros       */
+#define STEPQ_DEV_TIMEOUT 4u    /* a bounded device wait on a bulk copy gave up; head skipped      */
+
+/* ---- enumerations ------------------------------------------------------ */
+#define STEPQ_GATE_SCALAR 0     /* D = g I, one gate per (request, head)       (GDN) */
+#define STEPQ_GATE_DIAG 1       /* D = diag(g), one gate per key row           (KDA) */
+#define STEPQ_UNIT_HEAD 0       /* bit width chosen per head                         */
+#define STEPQ_UNIT_ROW 1        /* bit width chosen per key row                      */
+#define STEPQ_MODE_STEPQUANT 0  /* key-row-aware dual-axis fit (the method)          */
+#define STEPQ_MODE_UNIFORM 1    /* uniform INT-b comparator: per-row absmax, c = 1   */
+#define STEPQ_DTYPE_F32 0       /* q, k, v given as float32                          */
+#define STEPQ_DTYPE_BF16 1      /* q, k, v given as bfloat16                         */
+
+/*
+ * Plan description: what the offline lifetime-aware bit allocation and pivot
+ * selection hand to the runtime (hyper.ai summary, "Method": allocation and
+ * FP16 pivot selection run offline, so no per-token allocation cost), plus the
+ * calibrated row-impact weights (hyper.ai summary, "Method": row-impact score
+ * per key row).
+ *
+ *   d_k, d_v   state shape per head; this build runs d_k == d_v in {64, 128}
+ *              (others: STEPQ_ERR_UNSUPPORTED).
+ *   n_heads    heads per layer, >= 1.
+ *   gate_kind  STEPQ_GATE_SCALAR or STEPQ_GATE_DIAG.
+ *   unit_kind  STEPQ_UNIT_HEAD: bits has n_heads entries;
+ *              STEPQ_UNIT_ROW:  bits has n_heads * d_k entries.
+ *   mode       STEPQ_MODE_STEPQUANT or STEPQ_MODE_UNIFORM.
+ *   bits       host, per unit: 4, 6 or 8 (code width) or 16 (FP16 pivot).
+ *   w          host, [n_heads][d_k] row-impact weights, finite and > 0.
+ * Both arrays are copied; the caller keeps ownership.
+ */
+typedef struct stepq_plan_desc {
+    int32_t d_k;
+    int32_t d_v;
+    int32_t n_heads;
+    int32_t gate_kind;
+    int32_t unit_kind;
+    int32_t mode;
+    const uint8_t *bits;
+    const float *w;
+} stepq_plan_desc;
+
+typedef struct stepq_plan stepq_plan;
+typedef struct stepq_pool stepq_pool;
+
+/*
+ * Create a plan: validates the description, computes the packed byte layout
+ * of one slot and uploads the per-head / per-row tables to the current device.
+ *
+ * Layout of one slot (the pages give no byte format; this is the build's):
+ * the heads' blobs in head order, each starting on a 16-byte boundary; the
+ * slot stride is their total rounded up to 256 bytes.  A head blob is its key
+ * rows in ascending order -- a b-bit row holds d_v codes stored as
+ * code + 2^(b-1) in b bits each, LSB-first in the row's little-endian bit
+ * string; an FP16 pivot row holds d_v halves -- followed by rho[d_k] and
+ * c[d_v] as little-endian IEEE halves.  A head whose unit is an FP16 pivot is
+ * d_k*d_v halves, row-major, with no scales.
+ *
+ * Ownership: the plan is library-owned; release with stepq_plan_destroy.
+ * Errors: STEPQ_ERR_INVALID (bad description), STEPQ_ERR_UNSUPPORTED (shape),
+ * STEPQ_ERR_CUDA (device allocation / copy failed).
+ */
+STEPQ_API int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out);
+STEPQ_API int stepq_plan_destroy(stepq_plan *plan);
+
+/* Bytes of one slot (the pool's stride). */
+STEPQ_API int stepq_plan_slot_bytes(const stepq_plan *plan, size_t *out);
+
+/* Byte offset and size of head `head`'s blob inside a slot. */
+STEPQ_API int stepq_plan_head_layout(const stepq_plan *plan, int32_t head, size_t *offset,
+                                     size_t *bytes);
+
+/*
+ * Pool: a view over caller-owned device memory holding num_slots slots, one
+ * per concurrent request ("integrated into the recurrent state pool", hyper.ai
+ * summary, "Method", last paragraph).
+ *   dev_buf    device, >= num_slots * slot_bytes bytes, 256-byte aligned.
+ * The library allocates a 4-byte device status word and two CUDA events for
+ * the pool; stepq_pool_free releases those, never dev_buf.
+ * Errors: STEPQ_ERR_INVALID (NULL, too small, misaligned), STEPQ_ERR_CUDA.
+ */
+STEPQ_API int stepq_pool_alloc(const stepq_plan *plan, int64_t num_slots, void *dev_buf,
+                               size_t buf_bytes, stepq_pool **out);
+STEPQ_API int stepq_pool_free(stepq_pool *pool);
+
+/*
+ * Pack: quantise the given states X and write them into slots (admitting a
+ * request's state into the pool).  The quantiser is the one the decode step
+ * applies to the updated state (rcap.io post, decode-step pseudocode, last
+ * three lines).
+ *   slot_idx  device int32 [n], distinct, in [0, num_slots).
+ *   X         device float32 [n][n_heads][d_k][d_v].
+ */
+STEPQ_API int stepq_pack(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_idx,
+                         int64_t n, const float *X, void *stream);
+
+/*
+ * Unpack: reconstruct S = codes (.) (r c^T) (pivots raw) of the given slots
+ * (rcap.io post, decode-step pseudocode, first line).
+ *   S_out     device float32 [n][n_heads][d_k][d_v].
+ */
+STEPQ_API int stepq_unpack(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_idx,
+                           int64_t n, float *S_out, void *stream);
+
+/* Device workspace the decode step needs for n requests (the delta vector
+ * handed from the readout kernel to the fit kernel): n * n_heads * d_v floats. */
+STEPQ_API int stepq_workspace_bytes(const stepq_plan *plan, int64_t n, size_t *out);
+
+/*
+ * Readout half of the step (the fused kernel of hyper.ai summary, "Method",
+ * last paragraph): per (request, head) it reconstructs the packed state,
+ * forms u = (D S)^T k, delta = beta (v - u), and writes
+ * y = X^T q = (D S)^T q + (k.q) delta with X = D S + k delta^T (the gated
+ * Delta update, rcap.io post, decode-step pseudocode, lines 2-3).
+ *   qkv_dtype STEPQ_DTYPE_F32 or STEPQ_DTYPE_BF16.
+ *   q, k      device [n][n_heads][d_k];  v device [n][n_heads][d_v].
+ *   beta      device float32 [n][n_heads].
+ *   gate      device float32 [n][n_heads] (scalar) or [n][n_heads][d_k] (diag).
+ *   y         device float32 [n][n_heads][d_v] (written).
+ *   workspace device, >= stepq_workspace_bytes(n); delta is written there.
+ * The slots are only read.
+ */
+STEPQ_API int stepq_decode_readout(const stepq_plan *plan, stepq_pool *pool,
+                                   const int32_t *slot_idx, int64_t n, int32_t qkv_dtype,
+                                   const void *q, const void *k, const void *v,
+                                   const float *beta, const float *gate, float *y,
+                                   void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Fit-and-pack half of the step (hyper.ai summary, "Method", last paragraph:
+ * key-row-aware dual-axis fitting and pack write-back): per (request, head) it
+ * rebuilds X = D S + k delta^T from the still-untouched packed state and the
+ * delta left in `workspace` by stepq_decode_readout, fits the row factors
+ * r_i = sqrt(max_j |X_ij|) / sqrt(w_i) and the column scales by the
+ * 8-candidate impact-weighted least-squares search, and writes the codes
+ * clamp(rne(X / (r c)), +-qmax) back into the same slot.
+ * Must run after the readout of the same step has finished (same stream, or
+ * an event); k, gate and workspace must still hold that step's values.
+ */
+STEPQ_API int stepq_decode_fitpack(const stepq_plan *plan, stepq_pool *pool,
+                                   const int32_t *slot_idx, int64_t n, int32_t qkv_dtype,
+                                   const void *k, const float *gate, void *workspace,
+                                   size_t ws_bytes, void *stream);
+
+/*
+ * One whole decode step: readout on `main_stream`, then -- after an event --
+ * fit + pack on `side_stream`, so the caller's later work on `main_stream`
+ * (the next layer) overlaps the requantisation (hyper.ai summary, "Method",
+ * last paragraph; rcap.io post, "Calibration" paragraph).  y is ready in
+ * stream order on main_stream.  The call first makes main_stream wait for the
+ * previous step's fit on this pool, so back-to-back steps are safe.  With
+ * side_stream == main_stream (or NULL) both halves run on main_stream.
+ * Arguments as for the two halves.  Slots must be distinct within one call.
+ */
+STEPQ_API int stepq_decode_step(const stepq_plan *plan, stepq_pool *pool,
+                                const int32_t *slot_idx, int64_t n, int32_t qkv_dtype,
+                                const void *q, const void *k, const void *v, const float *beta,
+                                const float *gate, float *y, void *workspace, size_t ws_bytes,
+                                void *main_stream, void *side_stream);
+
+/*
+ * The unquantised baseline: the same gated Delta update and readout on an
+ * fp32 state pool, read and written in full (the FP32-state update the pages
+ * compare against, rcap.io post, results paragraph).
+ *   S          device float32 [num_slots][n_heads][d_k][d_v], updated in place.
+ *   dev_status device uint32 word for STEPQ_DEV_BAD_SLOT, or NULL.
+ * Other arguments as for stepq_decode_readout.
+ */
+STEPQ_API int stepq_fp32_step(int32_t d_k, int32_t d_v, int32_t n_heads, int32_t gate_kind,
+                              int32_t qkv_dtype, float *S, int64_t num_slots,
+                              const int32_t *slot_idx, int64_t n, const void *q, const void *k,
+                              const void *v, const float *beta, const float *gate, float *y,
+                              uint32_t *dev_status, void *stream);
+
+/* Synchronously read the pool's device status word (STEPQ_DEV_* bits, OR-ed
+ * over every call since the last clear).  Waits for the device to go idle. */
+STEPQ_API int stepq_get_status(stepq_pool *pool, uint32_t *out);
+
+/* Reset the pool's status word to 0, in stream order. */
+STEPQ_API int stepq_clear_status(stepq_pool *pool, void *stream);
+
+/* Message for the last failing call on this thread ("" if none). */
+STEPQ_API const char *stepq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STEPQ_H */

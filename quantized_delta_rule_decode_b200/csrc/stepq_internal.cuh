@@ -1,0 +1,66 @@
+// Internal definitions shared by the host API and the kernels of libstepq.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/stepq.h"
+
+namespace stepq {
+
+// How a head is stored.
+enum : uint8_t {
+    HK_UNIFORM = 0,  // every key row quantised at one width (head units)
+    HK_MIXED = 1,    // per-key-row widths, possibly with FP16 pivot rows (row units)
+    HK_PIVOT = 2,    // the whole head is an FP16 pivot: d_k*d_v raw halves
+};
+
+// Device-side view of a plan; passed by value to every kernel.
+struct PlanDev {
+    int dk, dv, H, gate_kind, unit_kind, mode;
+    uint32_t slot_bytes;
+    uint32_t max_head_bytes;
+    const uint32_t *head_off;    // [H] byte offset of the head blob in a slot
+    const uint32_t *head_bytes;  // [H] blob size (multiple of 16)
+    const uint32_t *scale_off;   // [H] offset of rho[dk]; c[dv] follows
+    const uint8_t *head_kind;    // [H] HK_*
+    const uint8_t *head_bits;    // [H] width of a HK_UNIFORM head
+    const uint8_t *row_bits;     // [H*dk] 4/6/8/16
+    const uint16_t *row_off;     // [H*dk] offset of the row inside the blob
+    const float *w;              // [H*dk] row-impact weights
+    const float *kappa;          // [H*dk] qmax_hi / qmax_i (1 for one-width heads)
+    const float *qmax_hi;        // [H] largest qmax over the head's quantised rows
+};
+
+// Everything a decode / pack launch needs besides the plan.
+struct StepArgs {
+    const uint8_t *pool_ro;
+    uint8_t *pool;
+    int64_t num_slots;
+    const int32_t *slot_idx;
+    int64_t n;
+    const void *q, *k, *v;
+    const float *beta, *gate;
+    float *y;
+    float *delta;      // workspace [n][H][dv]
+    const float *X;    // pack input [n][H][dk][dv]
+    float *S_out;      // unpack output
+    uint32_t *status;
+};
+
+// ---- launchers (stepq_kernels.cu) ------------------------------------------
+cudaError_t launch_readout(const PlanDev &P, const StepArgs &a, int qkv_dtype, cudaStream_t s);
+cudaError_t launch_fitpack(const PlanDev &P, const StepArgs &a, int qkv_dtype, cudaStream_t s);
+cudaError_t launch_pack(const PlanDev &P, const StepArgs &a, cudaStream_t s);
+cudaError_t launch_unpack(const PlanDev &P, const StepArgs &a, cudaStream_t s);
+cudaError_t launch_fp32_step(int d, int H, int gate_kind, int qkv_dtype, float *S, int64_t num_slots,
+                             const int32_t *slot_idx, int64_t n, const void *q, const void *k,
+                             const void *v, const float *beta, const float *gate, float *y,
+                             uint32_t *status, cudaStream_t s);
+
+size_t readout_smem_bytes(int d, uint32_t max_head_bytes);
+size_t quant_smem_bytes(int d, uint32_t max_head_bytes);
+
+}  // namespace stepq
