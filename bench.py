@@ -1,0 +1,640 @@
+#!/usr/bin/env python
+"""Throughput of the quantised gated Delta-rule decode step on B200.
+
+A *step* is one decode step of one linear-attention layer for a batch of
+requests: for every (request, head) read the packed state, reconstruct it,
+apply the gated Delta update, emit y = X^T q, refit the scales and write the
+state back packed (readout kernel on the main stream, fit + pack kernel on a
+second stream).  The metric is head-updates per second (one head-update = one
+(request, head) state step), plus the HBM bandwidth this implies.
+
+Default workload (fits one GPU): 64 requests x 32 heads, d_k = d_v = 128,
+bf16 q/k/v, scalar gates, per-head 4/6/8-bit plan averaging 6 bits plus one
+FP16 pivot head.  Inputs are synthetic and seeded (``workload.py``).
+
+Consecutive steps cycle through several layers' state pools whose total size
+is at least twice the 126 MB L2, so every step reads its state from HBM; as
+in a model, layer l's fit + pack overlaps layer l+1's readout.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl stepq|reference]
+Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
+GPU (weak scaling; the step has no cross-GPU exchange) and rank 0 prints one
+JSON line with the whole-job throughput, timed on the device as the max over
+ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workload as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+SMS, FP32_LANES = 148, 128
+METRIC = "quantized state-step throughput (head-updates/s) and HBM GB/s vs B200 peak"
+UNIT = "head-updates/s"
+ALU_OPS_PER_ENTRY = 60     # fp32 ops per quantised state entry in the fit + pack kernel
+PIVOT_OPS_PER_ENTRY = 6
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["stepq", "reference"], default="stepq")
+    ap.add_argument("--config", choices=W.CONFIG_ORDER, default="gdn")
+    ap.add_argument("--mode", choices=["stepquant", "uniform8", "uniform6"], default="stepquant")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--fp32-steps", type=int, default=2000)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--serial", action="store_true",
+                    help="also time the step with both kernels on one stream, one layer")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self, n):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            import torch
+            self.pg.barrier(device_ids=[self.local])
+            torch.cuda.synchronize()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+        self.idx = gpu_index
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                       "-i", str(gpu_index), "-lms", "100"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# ---------------------------------------------------------------------------
+# the workload on the device
+# ---------------------------------------------------------------------------
+def algorithmic_bytes(cfg, pin, slot_bytes_per_head):
+    """Bytes one step must move: packed state read + written, q,k,v, beta, gate, y."""
+    d = cfg.d
+    per_req = 2 * sum(slot_bytes_per_head)
+    qkv = 3 * d * (2 if cfg.bf16_inputs else 4)
+    gate = 4 * d if cfg.gate_kind == W.GATE_DIAG else 4
+    per_head_io = qkv + 4 + gate + 4 * d
+    return cfg.requests * (per_req + cfg.heads * per_head_io)
+
+
+def readout_bytes(cfg, slot_bytes_per_head):
+    d = cfg.d
+    qkv = 3 * d * (2 if cfg.bf16_inputs else 4)
+    gate = 4 * d if cfg.gate_kind == W.GATE_DIAG else 4
+    return cfg.requests * (sum(slot_bytes_per_head) + cfg.heads * (qkv + 4 + gate + 4 * d))
+
+
+def fit_alu_ops(cfg, pin):
+    d = cfg.d
+    if cfg.unit_kind == W.UNIT_HEAD:
+        q_rows = sum(d for b in pin.bits if b != 16)
+        p_rows = sum(d for b in pin.bits if b == 16)
+    else:
+        q_rows = int(np.sum(pin.bits != 16))
+        p_rows = int(np.sum(pin.bits == 16))
+    return cfg.requests * d * (q_rows * ALU_OPS_PER_ENTRY + p_rows * PIVOT_OPS_PER_ENTRY)
+
+
+class DeviceWorkload:
+    def __init__(self, cfg, mode):
+        import torch
+
+        import quantized_delta_rule_decode_b200 as S
+        self.S, self.cfg = S, cfg
+        ub = {"stepquant": None, "uniform8": 8, "uniform6": 6}[mode]
+        self.mode = W.MODE_UNIFORM if ub else W.MODE_STEPQUANT
+        self.pin = W.make_plan(cfg, uniform_bits=ub)
+        d, H, R = cfg.d, cfg.heads, cfg.requests
+        self.plan = S.stepq_plan_create(d, d, H, cfg.gate_kind, cfg.unit_kind, self.mode,
+                                        self.pin.bits, self.pin.w)
+        self.slot_bytes = S.stepq_plan_slot_bytes(self.plan)
+        self.head_bytes = [S.stepq_plan_head_layout(self.plan, h)[1] for h in range(H)]
+        self.nslots = cfg.pool_slots
+        pool_bytes = self.nslots * self.slot_bytes
+        self.layers = max(1, math.ceil(2 * L2_BYTES / pool_bytes))
+        self.slots_np = W.slot_indices(cfg)
+        self.slots = torch.from_numpy(self.slots_np).cuda()
+        # pack S0 into layer 0, chunk by chunk, then copy into the other layers
+        self.pools = []
+        for layer in range(self.layers):
+            buf = torch.zeros(pool_bytes, dtype=torch.uint8, device="cuda")
+            self.pools.append(S.stepq_pool_alloc(self.plan, self.nslots, buf))
+        chunk = max(1, (256 << 20) // (H * d * d * 4))
+        for r0 in range(0, R, chunk):
+            rr = list(range(r0, min(R, r0 + chunk)))
+            X = torch.from_numpy(W.initial_state(cfg, rr)).cuda()
+            S.stepq_pack(self.plan, self.pools[0], self.slots[r0:r0 + len(rr)].contiguous(), X)
+            del X
+        for p in self.pools[1:]:
+            p.buf.copy_(self.pools[0].buf)
+        torch.cuda.synchronize()
+        # ring of fresh step inputs
+        self.ring = []
+        dt = torch.bfloat16 if cfg.bf16_inputs else torch.float32
+        for step in range(16):
+            si = W.step_inputs(cfg, step, self.pin)
+            self.ring.append(dict(
+                q=torch.from_numpy(si.q).to(dt).cuda(), k=torch.from_numpy(si.k).to(dt).cuda(),
+                v=torch.from_numpy(si.v).to(dt).cuda(), beta=torch.from_numpy(si.beta).cuda(),
+                gate=torch.from_numpy(si.gate).cuda(), host=si))
+        self.dtype_code = S.DTYPE_BF16 if cfg.bf16_inputs else S.DTYPE_F32
+        self.y = torch.empty((R, H, d), dtype=torch.float32, device="cuda")
+        # one delta workspace per layer: layer l's fit may still read it while
+        # layer l+1's readout runs
+        self.ws = [torch.empty(S.stepq_workspace_bytes(self.plan, R), dtype=torch.uint8, device="cuda")
+                   for _ in range(self.layers)]
+        self.main = torch.cuda.current_stream()
+        self.side = torch.cuda.Stream()
+        L = S.load_library()
+        self.L = L
+        P = ctypes.c_void_p
+        ms, ss = P(self.main.cuda_stream), P(self.side.cuda_stream)
+        sp = P(self.slots.data_ptr())
+        self.step_args, self.read_args, self.fit_args = [], [], []
+        for layer in range(self.layers):
+            wsp, wsb = P(self.ws[layer].data_ptr()), self.ws[layer].numel()
+            for t in self.ring:
+                common = (self.plan.handle, self.pools[layer].handle, sp, R, self.dtype_code)
+                io = (P(t["q"].data_ptr()), P(t["k"].data_ptr()), P(t["v"].data_ptr()),
+                      P(t["beta"].data_ptr()), P(t["gate"].data_ptr()), P(self.y.data_ptr()),
+                      wsp, wsb)
+                self.step_args.append(common + io + (ms, ss))
+                self.read_args.append(common + io + (ms,))
+                self.fit_args.append(common + (P(t["k"].data_ptr()), P(t["gate"].data_ptr()),
+                                               wsp, wsb, ss))
+
+    def args_index(self, step):
+        return (step % self.layers) * 16 + (step % 16)
+
+    def run_step(self, step):
+        rc = self.L.stepq_decode_step(*self.step_args[self.args_index(step)])
+        if rc:
+            raise RuntimeError(self.L.stepq_last_error().decode())
+
+    def run_step_timed(self, step, ev):
+        """Same work as run_step, with CUDA events around each kernel on its own stream."""
+        i = self.args_index(step)
+        ev[0].record(self.main)
+        if self.L.stepq_decode_readout(*self.read_args[i]):
+            raise RuntimeError(self.L.stepq_last_error().decode())
+        ev[1].record(self.main)
+        self.side.wait_event(ev[1])
+        ev[2].record(self.side)
+        if self.L.stepq_decode_fitpack(*self.fit_args[i]):
+            raise RuntimeError(self.L.stepq_last_error().decode())
+        ev[3].record(self.side)
+
+    def join(self):
+        self.main.wait_stream(self.side)
+
+
+def time_device(wl, steps, warmup, dist, clocks_gpu):
+    import torch
+    for s in range(warmup):
+        wl.run_step(s)
+    wl.join()
+    torch.cuda.synchronize()
+    stride = max(1, steps // 2000)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(0, steps, stride)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    clk = Clocks(clocks_gpu)
+    time.sleep(0.3)
+    start.record(wl.main)
+    for s in range(steps):
+        if s % stride == 0:
+            wl.run_step_timed(warmup + s, evs[s // stride])
+        else:
+            wl.run_step(warmup + s)
+    wl.join()
+    end.record(wl.main)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    dist.barrier()
+    ms = start.elapsed_time(end)
+    ms = dist.max(ms)
+    readout_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    fit_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    return ms, statistics.mean(readout_ms), statistics.mean(fit_ms), clocks
+
+
+def time_serial(wl, steps, warmup):
+    """Both kernels on one stream, one layer after another, no overlap."""
+    import torch
+    for s in range(warmup):
+        wl.run_step_timed(s, [torch.cuda.Event() for _ in range(4)])
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(wl.main)
+    for s in range(steps):
+        i = wl.args_index(warmup + s)
+        args = list(wl.step_args[i])
+        args[-1] = args[-2]   # side stream := main stream
+        wl.L.stepq_decode_step(*args)
+    b.record(wl.main)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def time_e2e(wl, steps, warmup):
+    """Through the C ABI with host buffers: H2D of each step's inputs, the step, D2H of y."""
+    import torch
+    S, cfg = wl.S, wl.cfg
+    R, H, d = cfg.requests, cfg.heads, cfg.d
+    dt = torch.bfloat16 if cfg.bf16_inputs else torch.float32
+    ring = []
+    for t in wl.ring:
+        si = t["host"]
+        ring.append(dict(q=torch.from_numpy(si.q).to(dt).pin_memory(),
+                         k=torch.from_numpy(si.k).to(dt).pin_memory(),
+                         v=torch.from_numpy(si.v).to(dt).pin_memory(),
+                         beta=torch.from_numpy(si.beta).pin_memory(),
+                         gate=torch.from_numpy(si.gate).pin_memory()))
+    y = torch.empty((R, H, d), dtype=torch.float32).pin_memory()
+    # staging per layer: a layer's fit reads k and gate from it after the call returns
+    wss = [torch.empty(S.stepq_host_workspace_bytes(wl.plan, R, wl.dtype_code), dtype=torch.uint8,
+                       device="cuda") for _ in range(wl.layers)]
+    P = ctypes.c_void_p
+    args = []
+    for layer in range(wl.layers):
+        ws = wss[layer]
+        for t in ring:
+            args.append((wl.plan.handle, wl.pools[layer].handle, P(wl.slots.data_ptr()), R, wl.dtype_code,
+                         P(t["q"].data_ptr()), P(t["k"].data_ptr()), P(t["v"].data_ptr()),
+                         P(t["beta"].data_ptr()), P(t["gate"].data_ptr()), P(y.data_ptr()),
+                         P(ws.data_ptr()), ws.numel(), P(wl.main.cuda_stream),
+                         P(wl.side.cuda_stream)))
+    for s in range(warmup):
+        wl.L.stepq_decode_step_host(*args[wl.args_index(s)])
+    wl.join()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(wl.main)
+    for s in range(steps):
+        if wl.L.stepq_decode_step_host(*args[wl.args_index(warmup + s)]):
+            raise RuntimeError(wl.L.stepq_last_error().decode())
+    wl.join()
+    b.record(wl.main)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    t0 = ring[0]
+    h2d = sum(t0[k].numel() * t0[k].element_size() for k in ("q", "k", "v", "beta", "gate"))
+    d2h = y.numel() * y.element_size()
+    return ms, h2d, d2h
+
+
+def time_fp32(cfg, pin, steps, warmup):
+    import torch
+
+    import quantized_delta_rule_decode_b200 as S
+    d, H, R = cfg.d, cfg.heads, cfg.requests
+    per_layer = cfg.pool_slots * H * d * d * 4
+    layers = max(1, math.ceil(2 * L2_BYTES / per_layer))
+    if layers * per_layer > 40e9:
+        return None
+    pools = [torch.zeros((cfg.pool_slots, H, d, d), dtype=torch.float32, device="cuda") for _ in range(layers)]
+    slots = torch.from_numpy(W.slot_indices(cfg)).cuda()
+    dt = torch.bfloat16 if cfg.bf16_inputs else torch.float32
+    si = W.step_inputs(cfg, 0, pin)
+    q, k, v = (torch.from_numpy(a).to(dt).cuda() for a in (si.q, si.k, si.v))
+    beta, gate = torch.from_numpy(si.beta).cuda(), torch.from_numpy(si.gate).cuda()
+    y = torch.empty((R, H, d), dtype=torch.float32, device="cuda")
+    L = S.load_library()
+    P = ctypes.c_void_p
+    st = torch.cuda.current_stream()
+    code = S.DTYPE_BF16 if cfg.bf16_inputs else S.DTYPE_F32
+    args = [(d, d, H, cfg.gate_kind, code, P(p.data_ptr()), cfg.pool_slots, P(slots.data_ptr()), R,
+             P(q.data_ptr()), P(k.data_ptr()), P(v.data_ptr()), P(beta.data_ptr()),
+             P(gate.data_ptr()), P(y.data_ptr()), None, P(st.cuda_stream)) for p in pools]
+    for s in range(warmup):
+        L.stepq_fp32_step(*args[s % layers])
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for s in range(steps):
+        L.stepq_fp32_step(*args[s % layers])
+    b.record(st)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    qkv = 3 * d * (2 if cfg.bf16_inputs else 4)
+    gate_b = 4 * d if cfg.gate_kind == W.GATE_DIAG else 4
+    bytes_step = R * H * (2 * d * d * 4 + qkv + 4 + gate_b + 4 * d)
+    del pools
+    return {"value": R * H / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "hbm_gbs": bytes_step / (ms * 1e-3) / 1e9, "bytes_per_step": bytes_step, "layers": layers}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (reference arm / cpu_baseline)
+# ---------------------------------------------------------------------------
+class OracleRunner:
+    """The oracle as it stands: one (request, head) step per call, spread over host threads."""
+
+    def __init__(self, cfg, mode):
+        import oracle
+        ub = {"stepquant": None, "uniform8": 8, "uniform6": 6}[mode]
+        m = W.MODE_UNIFORM if ub else W.MODE_STEPQUANT
+        self.cfg = cfg
+        self.pin = W.make_plan(cfg, uniform_bits=ub)
+        self.plan = oracle.Plan(cfg.d, cfg.d, cfg.heads, cfg.gate_kind, cfg.unit_kind, m,
+                                self.pin.bits, self.pin.w)
+        self.threads = os.cpu_count() or 1
+        self.R = min(cfg.requests, max(2, self.threads))
+        X = W.initial_state(cfg, range(self.R))
+        self.blobs = {}
+        for r in range(self.R):
+            for h in range(cfg.heads):
+                blob, _ = self.plan.quantize_head(h, X[r, h])
+                self.blobs[(r, h)] = blob
+        self.si = W.step_inputs(cfg, 0, self.pin, range(self.R))
+        self.keys = list(self.blobs)
+        self.cursor = 0
+        from concurrent.futures import ThreadPoolExecutor
+        self.ex = ThreadPoolExecutor(self.threads)
+
+    def _one(self, key):
+        r, h = key
+        si = self.si
+        self.plan.step_head(h, self.blobs[key], si.q[r, h], si.k[r, h], si.v[r, h], si.beta[r, h],
+                            si.gate[r, h])
+
+    def run(self, count):
+        keys = [self.keys[(self.cursor + i) % len(self.keys)] for i in range(count)]
+        self.cursor += count
+        # each key at most once per batch: distinct blobs per concurrent call
+        for i in range(0, len(keys), len(self.keys)):
+            list(self.ex.map(self._one, keys[i:i + len(self.keys)]))
+
+    def rate(self, seconds):
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < seconds:
+            self.run(self.threads)
+            n += self.threads
+        return n / (time.perf_counter() - t0), n
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_reference(args, dist):
+    if dist.rank != 0:
+        return
+    cfg = W.CONFIGS[args.config]
+    orc = OracleRunner(cfg, args.mode)
+    warm_rate, _ = orc.rate(2.0)
+    budget = 150.0
+    per_step = int(max(1, min(cfg.requests * cfg.heads,
+                              budget * warm_rate / max(1, args.steps + args.warmup))))
+    steps = args.steps
+    if (args.steps + args.warmup) * per_step / warm_rate > budget * 1.5:
+        steps = max(1, int(budget * warm_rate / per_step) - args.warmup)
+    for _ in range(args.warmup):
+        orc.run(per_step)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        orc.run(per_step)
+    dt = time.perf_counter() - t0
+    value = steps * per_step / dt
+    sample = (f"{per_step} (request, head) oracle steps per timed step ({args.config} workload, "
+              f"{orc.R} requests x {cfg.heads} heads cycled), {steps} steps on {orc.threads} host threads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": dt / steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": workload_config(cfg, args.mode, None),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.threads, "kind": "oracle",
+                             "sample": sample, "cpu": cpu_model()},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg, mode, wl):
+    pin = wl.pin if wl is not None else W.make_plan(cfg)
+    counts = {int(b): int(np.sum(pin.bits == b)) for b in (4, 6, 8, 16) if np.sum(pin.bits == b)}
+    c = {"workload": f"{cfg.name}: {cfg.requests} requests x {cfg.heads} heads, d_k=d_v={cfg.d}, "
+                     f"{'KDA per-key-row' if cfg.gate_kind else 'GDN scalar'} gates, "
+                     f"{'bf16' if cfg.bf16_inputs else 'fp32'} q/k/v, 1 decode step per call",
+         "requests": cfg.requests, "heads": cfg.heads, "d_k": cfg.d, "d_v": cfg.d,
+         "quantizer": mode, "unit": "key row" if cfg.unit_kind else "head",
+         "plan_units_by_bits": counts, "global_batch": cfg.requests, "seq_len": 1,
+         "parallelism": "replicas (weak scaling)"}
+    if wl is not None:
+        c.update({"slot_bytes": wl.slot_bytes, "compression_vs_fp32": W.fp32_state_bytes(cfg) / wl.slot_bytes,
+                  "layer_pools_cycled": wl.layers,
+                  "l2": f"inputs larger than L2: {wl.layers} layer pools x "
+                        f"{wl.nslots * wl.slot_bytes / 1e6:.1f} MB cycled, no flush",
+                  "streams": "readout on main stream, fit+pack on a side stream; "
+                             "a layer's fit overlaps the next layer's readout"})
+    return c
+
+
+def src_sha():
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.join(ROOT, "quantized_delta_rule_decode_b200", "csrc"))):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(ROOT, "quantized_delta_rule_decode_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path)).get(kernel, {})
+    except (OSError, ValueError):
+        return None
+    if rec.get("src_sha") != src_sha() or rec.get("workload") != workload:
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def main():
+    args = parse()
+    dist = Dist(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, dist)
+        dist.close()
+        return
+    import torch
+    torch.cuda.set_device(dist.local)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    cfg = W.CONFIGS[args.config]
+    if args.steps < 1 or args.warmup < 3:
+        raise SystemExit("need --steps >= 1 and --warmup >= 3")
+
+    wl = DeviceWorkload(cfg, args.mode)
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_index = cvd.split(",")[dist.local].strip() if cvd else str(dist.local)
+    ms, readout_ms, fit_ms, clocks = time_device(wl, args.steps, args.warmup, dist, gpu_index)
+    ms_step = ms / args.steps
+    hu = dist.world * cfg.requests * cfg.heads
+    value = hu / (ms_step * 1e-3)
+    alg_bytes = algorithmic_bytes(cfg, wl.pin, wl.head_bytes)
+    hbm_gbs = dist.world * alg_bytes / (ms_step * 1e-3) / 1e9
+
+    rd_bytes = readout_bytes(cfg, wl.head_bytes)
+    rd_gbs = rd_bytes / (readout_ms * 1e-3) / 1e9
+    ops = fit_alu_ops(cfg, wl.pin)
+    clk_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+    alu_peak = SMS * FP32_LANES * clk_mhz * 1e6 / 1e12   # T fp32 lane-ops/s
+    fit_tops = ops / (fit_ms * 1e-3) / 1e12
+    kern = {"readout": {"us": readout_ms * 1e3, "bytes": rd_bytes, "gbs": rd_gbs,
+                        "frac_hbm": rd_gbs / hbm_peak},
+            "fitpack": {"us": fit_ms * 1e3, "fp32_ops": ops, "tops": fit_tops, "frac_alu": fit_tops / alu_peak}}
+    if fit_ms >= readout_ms:
+        roof = {"kernel": "fitpack (k_quant, fit+pack)", "bound": "alu", "achieved": fit_tops,
+                "peak": alu_peak, "unit": "T fp32 lane-ops/s", "frac": fit_tops / alu_peak,
+                "traffic": ncu_traffic("fitpack", cfg.name),
+                "peak_source": f"derived: {SMS} SMs x {FP32_LANES} FP32 lanes x {clk_mhz:.0f} MHz"}
+    else:
+        roof = {"kernel": "readout (k_readout)", "bound": "hbm", "achieved": rd_gbs, "peak": hbm_peak,
+                "unit": "GB/s", "frac": rd_gbs / hbm_peak, "traffic": ncu_traffic("readout", cfg.name),
+                "peak_source": peak_src}
+
+    serial = None
+    if args.serial and dist.world == 1:
+        sm = time_serial(wl, min(args.steps, 5000), args.warmup)
+        serial = {"ms_per_step": sm / min(args.steps, 5000)}
+    e2e_ms, h2d, d2h = time_e2e(wl, args.e2e_steps, max(3, args.warmup // 5))
+    e2e_ms = dist.max(e2e_ms)
+    e2e_value = hu / (e2e_ms / args.e2e_steps * 1e-3)
+    fp32 = time_fp32(cfg, wl.pin, args.fp32_steps, 10)
+    if fp32 is not None:
+        fp32["frac_hbm"] = fp32["hbm_gbs"] / hbm_peak
+        fp32["value"] *= dist.world
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
+        orc = OracleRunner(cfg, args.mode)
+        rate, n = orc.rate(args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": orc.threads, "kind": "oracle",
+               "sample": f"{n} (request, head) oracle steps of the {cfg.name} workload "
+                         f"({orc.R} requests x {cfg.heads} heads cycled) in {args.cpu_seconds:.0f} s",
+               "cpu": cpu_model()}
+
+    if dist.rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded; workload.py)",
+                "config": workload_config(cfg, args.mode, wl),
+                "hbm_gbs": hbm_gbs, "hbm_frac": hbm_gbs / hbm_peak, "hbm_peak_gbs": hbm_peak,
+                "hbm_peak_source": peak_src, "bytes_per_step": alg_bytes,
+                "roofline": roof, "kernels": kern,
+                "fp32_state_baseline": fp32,
+                "serial_step": serial,
+                "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps,
+                        "path": "stepq_decode_step_host (pinned host q,k,v,beta,gate in, y out)"},
+                "gpu_launches": 2 * args.steps,
+                "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()

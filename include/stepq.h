@@ -146,8 +146,8 @@ STEPQ_API int stepq_pool_free(stepq_pool *pool);
 /*
  * Pack: quantise the given states X and write them into slots (admitting a
  * request's state into the pool).  The quantiser is the one the decode step
- * applies to the updated state (rcap.io post, decode-step pseudocode, last
- * three lines).
+ * applies to the updated state (rcap.io post, decode-step pseudocode, the
+ * scale-fitting and quantise steps).
  *   slot_idx  device int32 [n], distinct, in [0, num_slots).
  *   X         device float32 [n][n_heads][d_k][d_v].
  */
@@ -156,7 +156,7 @@ STEPQ_API int stepq_pack(const stepq_plan *plan, stepq_pool *pool, const int32_t
 
 /*
  * Unpack: reconstruct S = codes (.) (r c^T) (pivots raw) of the given slots
- * (rcap.io post, decode-step pseudocode, first line).
+ * (rcap.io post, decode-step pseudocode, its unpack step).
  *   S_out     device float32 [n][n_heads][d_k][d_v].
  */
 STEPQ_API int stepq_unpack(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_idx,
@@ -171,7 +171,7 @@ STEPQ_API int stepq_workspace_bytes(const stepq_plan *plan, int64_t n, size_t *o
  * last paragraph): per (request, head) it reconstructs the packed state,
  * forms u = (D S)^T k, delta = beta (v - u), and writes
  * y = X^T q = (D S)^T q + (k.q) delta with X = D S + k delta^T (the gated
- * Delta update, rcap.io post, decode-step pseudocode, lines 2-3).
+ * Delta update, rcap.io post, decode-step pseudocode, its update and readout steps).
  *   qkv_dtype STEPQ_DTYPE_F32 or STEPQ_DTYPE_BF16.
  *   q, k      device [n][n_heads][d_k];  v device [n][n_heads][d_v].
  *   beta      device float32 [n][n_heads].
@@ -211,12 +211,35 @@ STEPQ_API int stepq_decode_fitpack(const stepq_plan *plan, stepq_pool *pool,
  * previous step's fit on this pool, so back-to-back steps are safe.  With
  * side_stream == main_stream (or NULL) both halves run on main_stream.
  * Arguments as for the two halves.  Slots must be distinct within one call.
+ * The fit still reads k, gate and workspace after the call returns: do not
+ * overwrite them, or hand the same workspace to another pool's step, until
+ * side_stream has finished this step (one workspace per layer in flight).
  */
 STEPQ_API int stepq_decode_step(const stepq_plan *plan, stepq_pool *pool,
                                 const int32_t *slot_idx, int64_t n, int32_t qkv_dtype,
                                 const void *q, const void *k, const void *v, const float *beta,
                                 const float *gate, float *y, void *workspace, size_t ws_bytes,
                                 void *main_stream, void *side_stream);
+
+/*
+ * The same whole step for callers whose per-token inputs live in host memory
+ * (a C caller without a device allocator of its own for them): the call
+ * copies q, k, v, beta and gate host -> device into `workspace`, runs
+ * stepq_decode_step, and copies y device -> host, all in stream order on
+ * main_stream.  Host buffers should be pinned (cudaHostAlloc) for the copies
+ * to be asynchronous; y_host is valid once main_stream reaches that point.
+ *   q_host..gate_host, y_host: host, same shapes and types as for
+ *             stepq_decode_step.
+ *   workspace device, >= stepq_host_workspace_bytes(plan, n, qkv_dtype).
+ */
+STEPQ_API int stepq_host_workspace_bytes(const stepq_plan *plan, int64_t n, int32_t qkv_dtype,
+                                         size_t *out);
+STEPQ_API int stepq_decode_step_host(const stepq_plan *plan, stepq_pool *pool,
+                                     const int32_t *slot_idx, int64_t n, int32_t qkv_dtype,
+                                     const void *q_host, const void *k_host, const void *v_host,
+                                     const float *beta_host, const float *gate_host,
+                                     float *y_host, void *workspace, size_t ws_bytes,
+                                     void *main_stream, void *side_stream);
 
 /*
  * The unquantised baseline: the same gated Delta update and readout on an

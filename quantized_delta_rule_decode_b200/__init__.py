@@ -29,8 +29,10 @@ from ._ffi import (  # noqa: F401
     stepq_decode_fitpack,
     stepq_decode_readout,
     stepq_decode_step,
+    stepq_decode_step_host,
     stepq_fp32_step,
     stepq_get_status,
+    stepq_host_workspace_bytes,
     stepq_pack,
     stepq_plan_create,
     stepq_plan_destroy,

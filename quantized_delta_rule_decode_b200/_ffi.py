@@ -34,6 +34,8 @@ _SIGS = {
     "stepq_decode_step": [_P, _P, _P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P],
     "stepq_fp32_step": [_I32, _I32, _I32, _I32, _I32, _P, _I64, _P, _I64, _P, _P, _P, _P, _P, _P,
                         _P, _P],
+    "stepq_host_workspace_bytes": [_P, _I64, _I32, ctypes.POINTER(_SZ)],
+    "stepq_decode_step_host": [_P, _P, _P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P],
     "stepq_get_status": [_P, ctypes.POINTER(ctypes.c_uint32)],
     "stepq_clear_status": [_P, _P],
     "stepq_last_error": [],
@@ -236,6 +238,29 @@ def stepq_decode_step(plan, pool, slot_idx, q, k, v, beta, gate, y, workspace, m
     _call("stepq_decode_step", plan.handle, pool.handle, s, n, _qkv_dtype(q), _ptr(q, q.dtype, "q"),
           _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"), _ptr(beta, torch.float32, "beta"),
           _ptr(gate, torch.float32, "gate"), _ptr(y, torch.float32, "y"),
+          _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size(), m, sd)
+
+
+def stepq_host_workspace_bytes(plan: Plan, n: int, qkv_dtype: int) -> int:
+    out = _SZ()
+    _call("stepq_host_workspace_bytes", plan.handle, n, qkv_dtype, ctypes.byref(out))
+    return out.value
+
+
+def _hptr(t, name):
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def stepq_decode_step_host(plan, pool, slot_idx, q, k, v, beta, gate, y, workspace,
+                           main_stream=None, side_stream=None):
+    """q..gate and y are host (ideally pinned) tensors; workspace is on the device."""
+    s, n = _slots(slot_idx)
+    m = _stream(main_stream)
+    sd = _stream(side_stream) if side_stream is not None else m
+    _call("stepq_decode_step_host", plan.handle, pool.handle, s, n, _qkv_dtype(q), _hptr(q, "q"),
+          _hptr(k, "k"), _hptr(v, "v"), _hptr(beta, "beta"), _hptr(gate, "gate"), _hptr(y, "y"),
           _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size(), m, sd)
 
 

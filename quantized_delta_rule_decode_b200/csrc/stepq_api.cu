@@ -21,6 +21,8 @@ struct stepq_plan {
     std::vector<uint8_t> head_kind, head_bits, row_bits;
     std::vector<uint16_t> row_off;
     std::vector<float> w, kappa, qmax_hi;
+    std::vector<int16_t> qheads, pheads;
+    uint32_t max_qhead_bytes = 0;
     void *dev_tables = nullptr;
     stepq::PlanDev dev{};
 };
@@ -174,11 +176,13 @@ int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out) {
             p->kappa[(size_t)h * dk + i] =
                 b == 16 ? 0.0f : (float)qhi / (float)((1 << (b - 1)) - 1);
         }
+        p->scale_off[h] = (uint32_t)hb;
         if (pivot_head) {
-            p->scale_off[h] = (uint32_t)hb;
+            p->pheads.push_back((int16_t)h);
         } else {
-            p->scale_off[h] = (uint32_t)hb;
             hb += (size_t)dk * 2 + (size_t)dv * 2;
+            p->qheads.push_back((int16_t)h);
+            p->max_qhead_bytes = std::max<uint32_t>(p->max_qhead_bytes, (uint32_t)round_up(hb, 16));
         }
         hb = round_up(hb, 16);
         p->head_off[h] = (uint32_t)off;
@@ -197,7 +201,9 @@ int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out) {
     size_t o_head_off = 0, o_head_bytes = o_head_off + 4 * H, o_scale_off = o_head_bytes + 4 * H;
     size_t o_kind = o_scale_off + 4 * H, o_hbits = o_kind + H, o_rbits = o_hbits + H;
     size_t o_roff = round_up(o_rbits + HD, 16), o_w = round_up(o_roff + 2 * HD, 16);
-    size_t o_kap = o_w + 4 * HD, o_qhi = o_kap + 4 * HD, total = o_qhi + 4 * H;
+    size_t o_kap = o_w + 4 * HD, o_qhi = o_kap + 4 * HD;
+    size_t o_qh = round_up(o_qhi + 4 * H, 16), o_ph = round_up(o_qh + 2 * H, 16);
+    size_t total = o_ph + 2 * H;
     std::vector<uint8_t> host(total, 0);
     memcpy(&host[o_head_off], p->head_off.data(), 4 * H);
     memcpy(&host[o_head_bytes], p->head_bytes.data(), 4 * H);
@@ -209,6 +215,8 @@ int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out) {
     memcpy(&host[o_w], p->w.data(), 4 * HD);
     memcpy(&host[o_kap], p->kappa.data(), 4 * HD);
     memcpy(&host[o_qhi], p->qmax_hi.data(), 4 * H);
+    if (!p->qheads.empty()) memcpy(&host[o_qh], p->qheads.data(), 2 * p->qheads.size());
+    if (!p->pheads.empty()) memcpy(&host[o_ph], p->pheads.data(), 2 * p->pheads.size());
     cudaError_t e = cudaGetDevice(&p->device);
     if (e == cudaSuccess) e = cudaMalloc(&p->dev_tables, total);
     if (e == cudaSuccess) e = cudaMemcpy(p->dev_tables, host.data(), total, cudaMemcpyHostToDevice);
@@ -233,6 +241,11 @@ int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out) {
     v.w = reinterpret_cast<const float *>(t + o_w);
     v.kappa = reinterpret_cast<const float *>(t + o_kap);
     v.qmax_hi = reinterpret_cast<const float *>(t + o_qhi);
+    v.n_qheads = (int)p->qheads.size();
+    v.n_pheads = (int)p->pheads.size();
+    v.max_qhead_bytes = p->max_qhead_bytes;
+    v.qheads = reinterpret_cast<const int16_t *>(t + o_qh);
+    v.pheads = reinterpret_cast<const int16_t *>(t + o_ph);
     *out = p;
     return STEPQ_OK;
 }
@@ -419,6 +432,78 @@ int stepq_decode_step(const stepq_plan *plan, stepq_pool *pool, const int32_t *s
         if (e != cudaSuccess) return cuda_fail(e, "stream handoff");
     }
     return stepq_decode_fitpack(plan, pool, slot_idx, n, qkv_dtype, k, gate, workspace, ws_bytes, s);
+}
+
+namespace {
+struct HostLayout {
+    size_t delta, q, k, v, beta, gate, y, total, qkv_bytes, gate_bytes, y_bytes, beta_bytes;
+};
+HostLayout host_layout(const stepq_plan *plan, int64_t n, int32_t qkv_dtype) {
+    HostLayout L{};
+    const size_t nh = (size_t)n * plan->H;
+    const size_t es = qkv_dtype == STEPQ_DTYPE_BF16 ? 2 : 4;
+    L.qkv_bytes = nh * plan->dk * es;
+    L.beta_bytes = nh * 4;
+    L.gate_bytes = plan->gate_kind == STEPQ_GATE_DIAG ? nh * plan->dk * 4 : nh * 4;
+    L.y_bytes = nh * plan->dv * 4;
+    L.delta = 0;
+    L.q = round_up(nh * plan->dv * 4, 256);
+    L.k = L.q + round_up(L.qkv_bytes, 256);
+    L.v = L.k + round_up(L.qkv_bytes, 256);
+    L.beta = L.v + round_up(L.qkv_bytes, 256);
+    L.gate = L.beta + round_up(L.beta_bytes, 256);
+    L.y = L.gate + round_up(L.gate_bytes, 256);
+    L.total = L.y + round_up(L.y_bytes, 256);
+    return L;
+}
+}  // namespace
+
+int stepq_host_workspace_bytes(const stepq_plan *plan, int64_t n, int32_t qkv_dtype, size_t *out) {
+    if (!plan || !out) return fail(STEPQ_ERR_INVALID, "plan and out must be non-NULL");
+    if (n < 0) return fail(STEPQ_ERR_INVALID, "n must be >= 0");
+    if (qkv_dtype != STEPQ_DTYPE_F32 && qkv_dtype != STEPQ_DTYPE_BF16)
+        return fail(STEPQ_ERR_INVALID, "qkv_dtype %d unknown", qkv_dtype);
+    *out = host_layout(plan, n, qkv_dtype).total;
+    return STEPQ_OK;
+}
+
+int stepq_decode_step_host(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_idx,
+                           int64_t n, int32_t qkv_dtype, const void *q_host, const void *k_host,
+                           const void *v_host, const float *beta_host, const float *gate_host,
+                           float *y_host, void *workspace, size_t ws_bytes, void *main_stream,
+                           void *side_stream) {
+    g_err.clear();
+    int rc = check_pool(plan, pool);
+    if (!rc) rc = check_rows(plan, slot_idx, n);
+    if (rc) return rc;
+    if (n == 0) return STEPQ_OK;
+    if (qkv_dtype != STEPQ_DTYPE_F32 && qkv_dtype != STEPQ_DTYPE_BF16)
+        return fail(STEPQ_ERR_INVALID, "qkv_dtype %d unknown", qkv_dtype);
+    if (!q_host || !k_host || !v_host || !beta_host || !gate_host || !y_host)
+        return fail(STEPQ_ERR_INVALID, "host buffers must be non-NULL");
+    if ((rc = check_inputs(workspace, "workspace"))) return rc;
+    const HostLayout L = host_layout(plan, n, qkv_dtype);
+    if (ws_bytes < L.total)
+        return fail(STEPQ_ERR_INVALID, "workspace of %zu bytes, %zu needed", ws_bytes, L.total);
+    uint8_t *w = static_cast<uint8_t *>(workspace);
+    cudaStream_t m = static_cast<cudaStream_t>(main_stream);
+    // the staging area must not be overwritten while the previous step's fit
+    // (which reads k and gate from it) is still running
+    if ((rc = wait_pending_fit(pool, m))) return rc;
+    cudaError_t e = cudaMemcpyAsync(w + L.q, q_host, L.qkv_bytes, cudaMemcpyHostToDevice, m);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.k, k_host, L.qkv_bytes, cudaMemcpyHostToDevice, m);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.v, v_host, L.qkv_bytes, cudaMemcpyHostToDevice, m);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.beta, beta_host, L.beta_bytes, cudaMemcpyHostToDevice, m);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.gate, gate_host, L.gate_bytes, cudaMemcpyHostToDevice, m);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    rc = stepq_decode_step(plan, pool, slot_idx, n, qkv_dtype, w + L.q, w + L.k, w + L.v,
+                           reinterpret_cast<const float *>(w + L.beta),
+                           reinterpret_cast<const float *>(w + L.gate),
+                           reinterpret_cast<float *>(w + L.y), w + L.delta, L.q, main_stream,
+                           side_stream);
+    if (rc) return rc;
+    e = cudaMemcpyAsync(y_host, w + L.y, L.y_bytes, cudaMemcpyDeviceToHost, m);
+    return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "device-to-host copy");
 }
 
 int stepq_fp32_step(int32_t d_k, int32_t d_v, int32_t n_heads, int32_t gate_kind,

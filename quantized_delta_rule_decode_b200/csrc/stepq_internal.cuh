@@ -32,6 +32,10 @@ struct PlanDev {
     const float *w;              // [H*dk] row-impact weights
     const float *kappa;          // [H*dk] qmax_hi / qmax_i (1 for one-width heads)
     const float *qmax_hi;        // [H] largest qmax over the head's quantised rows
+    int n_qheads, n_pheads;      // quantised heads, FP16 pivot heads
+    uint32_t max_qhead_bytes;    // largest blob of a quantised (non-pivot) head
+    const int16_t *qheads;       // [n_qheads] indices of the quantised heads
+    const int16_t *pheads;       // [n_pheads] indices of the FP16 pivot heads
 };
 
 // Everything a decode / pack launch needs besides the plan.
@@ -61,6 +65,6 @@ cudaError_t launch_fp32_step(int d, int H, int gate_kind, int qkv_dtype, float *
                              uint32_t *status, cudaStream_t s);
 
 size_t readout_smem_bytes(int d, uint32_t max_head_bytes);
-size_t quant_smem_bytes(int d, uint32_t max_head_bytes);
+size_t quant_smem_bytes(int d, uint32_t max_qhead_bytes);
 
 }  // namespace stepq

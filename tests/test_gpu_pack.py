@@ -1,7 +1,7 @@
 """GPU pack / unpack vs the oracle, through the C ABI (bit-exact contract).
 
 Pack quantises a given X (the same quantiser the decode step applies to the
-updated state: rcap.io post, decode-step pseudocode, last three lines; the
+updated state: rcap.io post, decode-step pseudocode, its fit and quantise steps; the
 key-row-aware dual-axis fit of the hyper.ai summary, "Method").  From an
 identical X the packed bytes must equal the oracle's, except for a column
 whose argmin is a near tie (see gpu_harness.compare_pack).
