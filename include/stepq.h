@@ -255,6 +255,31 @@ STEPQ_API int stepq_fp32_step(int32_t d_k, int32_t d_v, int32_t n_heads, int32_t
                               const void *v, const float *beta, const float *gate, float *y,
                               uint32_t *dev_status, void *stream);
 
+/*
+ * The whole decode step with no device allocation anywhere: the same kernels
+ * and arguments as stepq_decode_step, minus the workspace.  (Not a step of
+ * the paper's method: it exists for callers that cannot allocate device
+ * memory -- a framework whose caching allocator owns all of it, a process
+ * that may not grow its device footprint after start-up, a C caller with no
+ * allocator.)  The delta vector handed from the readout to the fit kernel is
+ * kept in a fixed array inside the library's device image, 4 MiB on every
+ * GPU that loads the library, held until the process exits.
+ *   - n * n_heads * d_v must not exceed STEPQ_STATIC_DELTA_FLOATS, else
+ *     STEPQ_ERR_INVALID and nothing is launched.
+ *   - the first call on a device looks up the array's device address once
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - every call shares the one array: calls whose kernels can overlap on the
+ *     GPU (another stream, or the fit of the previous call on side_stream
+ *     still running when the next call's readout starts on a different pool)
+ *     race on it.  Serialise them, e.g. pass side_stream == main_stream.
+ */
+#define STEPQ_STATIC_DELTA_FLOATS 1048576
+STEPQ_API int stepq_decode_step_static(const stepq_plan *plan, stepq_pool *pool,
+                                       const int32_t *slot_idx, int64_t n, int32_t qkv_dtype,
+                                       const void *q, const void *k, const void *v,
+                                       const float *beta, const float *gate, float *y,
+                                       void *main_stream, void *side_stream);
+
 /* Synchronously read the pool's device status word (STEPQ_DEV_* bits, OR-ed
  * over every call since the last clear).  Waits for the device to go idle. */
 STEPQ_API int stepq_get_status(stepq_pool *pool, uint32_t *out);

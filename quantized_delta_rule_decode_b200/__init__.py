@@ -30,6 +30,7 @@ from ._ffi import (  # noqa: F401
     stepq_decode_readout,
     stepq_decode_step,
     stepq_decode_step_host,
+    stepq_decode_step_static,
     stepq_fp32_step,
     stepq_get_status,
     stepq_host_workspace_bytes,

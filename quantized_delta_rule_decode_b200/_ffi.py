@@ -36,6 +36,7 @@ _SIGS = {
                         _P, _P],
     "stepq_host_workspace_bytes": [_P, _I64, _I32, ctypes.POINTER(_SZ)],
     "stepq_decode_step_host": [_P, _P, _P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P],
+    "stepq_decode_step_static": [_P, _P, _P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P, _P],
     "stepq_get_status": [_P, ctypes.POINTER(ctypes.c_uint32)],
     "stepq_clear_status": [_P, _P],
     "stepq_last_error": [],
@@ -262,6 +263,22 @@ def stepq_decode_step_host(plan, pool, slot_idx, q, k, v, beta, gate, y, workspa
     _call("stepq_decode_step_host", plan.handle, pool.handle, s, n, _qkv_dtype(q), _hptr(q, "q"),
           _hptr(k, "k"), _hptr(v, "v"), _hptr(beta, "beta"), _hptr(gate, "gate"), _hptr(y, "y"),
           _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size(), m, sd)
+
+
+STATIC_DELTA_FLOATS = 1048576
+
+
+def stepq_decode_step_static(plan, pool, slot_idx, q, k, v, beta, gate, y, main_stream=None,
+                             side_stream=None):
+    """stepq_decode_step without a workspace (no device allocation anywhere)."""
+    import torch
+    s, n = _slots(slot_idx)
+    m = _stream(main_stream)
+    sd = _stream(side_stream) if side_stream is not None else m
+    _call("stepq_decode_step_static", plan.handle, pool.handle, s, n, _qkv_dtype(q),
+          _ptr(q, q.dtype, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"),
+          _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
+          _ptr(y, torch.float32, "y"), m, sd)
 
 
 def stepq_fp32_step(S, slot_idx, q, k, v, beta, gate, y, gate_kind, dev_status=None, stream=None):

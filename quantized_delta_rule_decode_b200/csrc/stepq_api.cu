@@ -112,6 +112,10 @@ int wait_pending_fit(stepq_pool *pool, cudaStream_t s) {
 
 }  // namespace
 
+namespace stepq {
+int set_error(int code, const char *msg) { return fail(code, "%s", msg); }
+}  // namespace stepq
+
 extern "C" {
 
 const char *stepq_last_error(void) { return g_err.c_str(); }
