@@ -9,8 +9,10 @@
  *
  * Arithmetic: IEEE binary32 (`float`) throughout, as the workloads fix ("fp32
  * state math"), round-to-nearest-even, compiled with -ffp-contract=off so no
- * multiply-add is fused.  Every sum runs over ascending index.  Code and
- * scale decisions are taken in that same binary32 arithmetic.
+ * multiply-add is fused unless written as fmaf().  Every sum runs over
+ * ascending index, except the column-fit objective, whose order is stated in
+ * objective().  Code and scale decisions are taken in that same binary32
+ * arithmetic.
  *
  * Sources (the pages, cited by title and part):
  *   [P1] hyper.ai summary of "STEPQuant: When and Where Errors Matter in
@@ -39,6 +41,10 @@
  *   - a zero row (max |X_ij| = 0) stores rho = 0 and codes 0 and takes no part
  *     in the column fit; a zero column stores c = 0; a row holding a NaN or an
  *     infinity is stored as a zero row and raises STATUS_NONFINITE.
+ *   - the column-fit objective sum_i w_i^2 (X_ij - r_i c code_ij)^2 is
+ *     evaluated in one stated binary32 order (see objective()), because the
+ *     argmin it feeds is an integer decision that the CUDA kernels must
+ *     reproduce exactly for multi-step rollouts to agree.
  *
  * Parity status of each function is stated in its comment ("pinned by ...").
  */
@@ -344,6 +350,39 @@ void orc_dequantize_head(const void *p, int h, const uint8_t *blob, float *S)
 
 static const float ALPHA[8] = {1.0f, 0.95f, 0.9f, 0.85f, 0.8f, 0.75f, 0.7f, 0.65f};
 
+/* The weighted least-squares objective of one candidate column scale c,
+ * E = sum_i w_i^2 (X_ij - r_i c code_i)^2, evaluated in units of each row's
+ * quantisation step: with z_i = |X_ij| * (1/r_i) and t_i = z_i * (1/c),
+ *     E = c^2 * sum_i A_i (t_i - code_i)^2,   A_i = (w_i r_i)^2,
+ * code_i = min(rne(t_i), qmax_i).  binary32, in this order:
+ *   - 1/r_i and 1/c correctly rounded; z_i = |X_ij| * (1/r_i) rounded;
+ *   - q = fmaf(z_i, 1/c, 2^23) rounds t_i to an integer (exact product,
+ *     one rounding); clamp q to 2^23 + qmax_i; d_i = fmaf(z_i, 1/c, 2^23 - q);
+ *   - four partial sums P_g over the rows i = g, g+4, g+8, ... (ascending),
+ *     P_g = fmaf(A_i * d_i, d_i, P_g);
+ *   - E = (c * c) * ((P_0 + P_1) + (P_2 + P_3)).
+ * Rows that are zero, non-finite or FP16 pivots take no part. */
+static float objective(const float *X, int dv, int j, int dk, const int *active,
+                       const float *irho, const float *A, const int *qmax, float c)
+{
+    const float two23 = 8388608.0f;
+    float ic = 1.0f / c;
+    float P[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    int i;
+    for (i = 0; i < dk; i++) {
+        float z, q, d;
+        if (!active[i])
+            continue;
+        z = fabsf(X[i * dv + j]) * irho[i];
+        q = fmaf(z, ic, two23);
+        if (q > two23 + (float)qmax[i])
+            q = two23 + (float)qmax[i];
+        d = fmaf(z, ic, two23 - q);
+        P[i & 3] = fmaf(A[i] * d, d, P[i & 3]);
+    }
+    return (c * c) * ((P[0] + P[1]) + (P[2] + P[3]));
+}
+
 static int code_of(float x, float P, int qmax)
 {
     float t = x / P;                              /* X / (r c), one rounding */
@@ -389,6 +428,8 @@ int orc_quantize_head(const void *p, int h, const float *X, uint8_t *blob,
     int *qmax = (int *)calloc(dk, sizeof(int));
     float *kappa = (float *)calloc(dk, sizeof(float));
     int16_t *col = (int16_t *)calloc(dk, sizeof(int16_t));
+    float *irho = (float *)calloc(dk, sizeof(float));
+    float *Aw = (float *)calloc(dk, sizeof(float));
     int qhi = 0;
 
     if (E_diag) for (a = 0; a < dv * 8; a++) E_diag[a] = 0.0f;
@@ -444,6 +485,13 @@ int orc_quantize_head(const void *p, int h, const float *X, uint8_t *blob,
             for (j = 0; j < dv; j++)
                 c[j] = 0x3c00;                    /* 1.0 */
         } else {
+            for (i = 0; i < dk; i++) {
+                if (!active[i])
+                    continue;
+                irho[i] = 1.0f / orc_half_to_float(rho[i]);
+                Aw[i] = (pl->w[h * dk + i] * orc_half_to_float(rho[i])) *
+                        (pl->w[h * dk + i] * orc_half_to_float(rho[i]));
+            }
             for (j = 0; j < dv; j++) {
                 float M = 0.0f, Ebest = 0.0f;
                 int best = 0;
@@ -461,19 +509,8 @@ int orc_quantize_head(const void *p, int h, const float *X, uint8_t *blob,
                 }
                 for (a = 0; a < 8; a++) {
                     uint16_t ca = scale_half((ALPHA[a] * M) / (float)qhi);
-                    float cf = orc_half_to_float(ca);
-                    float E = 0.0f;
-                    for (i = 0; i < dk; i++) {
-                        float P, e, wi;
-                        int code;
-                        if (!active[i])
-                            continue;
-                        P = orc_half_to_float(rho[i]) * cf;
-                        code = code_of(X[i * dv + j], P, qmax[i]);
-                        e = X[i * dv + j] - P * (float)code;
-                        wi = pl->w[h * dk + i];
-                        E = E + (wi * wi) * (e * e);
-                    }
+                    float E = objective(X, dv, j, dk, active, irho, Aw, qmax,
+                                        orc_half_to_float(ca));
                     if (E_diag) E_diag[j * 8 + a] = E;
                     if (cand_diag) cand_diag[j * 8 + a] = ca;
                     if (a == 0 || E < Ebest) {    /* strict: ties keep the larger alpha */
@@ -493,6 +530,7 @@ int orc_quantize_head(const void *p, int h, const float *X, uint8_t *blob,
     }
     orc_pack_codes(p, h, codes, piv, rho, c, blob);
     free(codes); free(piv); free(rho); free(c); free(active); free(qmax); free(kappa); free(col);
+    free(irho); free(Aw);
     return status;
 }
 

@@ -64,7 +64,6 @@ cudaError_t launch_fp32_step(int d, int H, int gate_kind, int qkv_dtype, float *
                              const void *v, const float *beta, const float *gate, float *y,
                              uint32_t *status, cudaStream_t s);
 
-size_t readout_smem_bytes(int d, uint32_t max_head_bytes);
 
 // Record an error message for stepq_last_error(); returns code.
 int set_error(int code, const char *msg);

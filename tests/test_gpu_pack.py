@@ -1,10 +1,11 @@
 """GPU pack / unpack vs the oracle, through the C ABI (bit-exact contract).
 
 Pack quantises a given X (the same quantiser the decode step applies to the
-updated state: rcap.io post, decode-step pseudocode, its fit and quantise steps; the
-key-row-aware dual-axis fit of the hyper.ai summary, "Method").  From an
-identical X the packed bytes must equal the oracle's, except for a column
-whose argmin is a near tie (see gpu_harness.compare_pack).
+updated state: rcap.io post, decode-step pseudocode, its fit and quantise
+steps; the key-row-aware dual-axis fit of the hyper.ai summary, "Method").
+From an identical X the packed bytes must equal the oracle's.  compare_pack
+would also accept an argmin that differs on a near tie (the general
+contract), and the tests then require that no column needed it.
 """
 
 import numpy as np
@@ -47,7 +48,10 @@ def test_pack_matches_oracle(name, mode, ub, R):
             compare_pack(pair, h, pair.head_blob(g, slots[r], h), pair.head_blob(o, slots[r], h),
                          X[r, h], stats)
     assert S.stepq_get_status(pool) == 0
-    assert stats["switched_cols"] <= 2, stats
+    # the kernels evaluate the column objective in the oracle's stated order,
+    # so even the argmin agrees: the bytes are identical
+    assert stats["switched_cols"] == 0, stats
+    assert np.array_equal(g, o)
 
 
 def test_pack_degenerate_values():

@@ -148,16 +148,18 @@ def _check_head(orc, plan, X, w, row_bits, stats):
                 q = max(-qmax[row_bits[i]], min(qmax[row_bits[i]], rne_int(t)))
                 e = Fr(float(X[i, j])) - P * q
                 e_sum += wF[i] * wF[i] * e * e
-                cancel += wF[i] * wF[i] * abs(e) * abs(P * q)
+                cancel += wF[i] * wF[i] * abs(e) * abs(Fr(float(X[i, j])))
             Ex.append(e_sum)
             if tie:
                 stats["code_tie"] += 1
             else:
-                # first-order bound of the binary32 evaluation: the sum of
-                # positive terms (dk+6 roundings) plus the cancellation in
-                # e = X - fl(P*code), which contributes 2u|e||P*code| per term
+                # first-order bound of the oracle's binary32 evaluation in
+                # step units (t = |X| (1/rho)(1/c), three roundings, so
+                # |dt| <= 3u t, and d^2 moves by <= 2|d| 3u t; in X units that
+                # is 6u w^2 |e||X| per term) plus the weights, products and
+                # the four partial sums (<= dk + 12 roundings of E)
                 u = Fr(1, 2 ** 24)
-                bound = (dk + 6) * u * e_sum + Fr(5, 2) * u * cancel
+                bound = (dk + 12) * u * e_sum + 8 * u * cancel
                 assert abs(Fr(float(E[j, a])) - e_sum) <= bound, (j, a)
         # ---- argmin, ties to the larger alpha (first index) ----
         eb = min(Ex)
