@@ -1,0 +1,79 @@
+"""Multi-rank host logic on CPU (gloo, world size 2).
+
+The decode step shards across GPUs with no exchange: every (request, head)
+update is independent (rcap.io post: a fixed-size state per request per
+head).  Ranks that each step their own requests reproduce a single-process
+step exactly, and bench.py's ranks meet only at the timing barrier and the
+max-over-ranks reduction, exercised here with gloo.
+"""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+import oracle
+import workload as W
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, q):
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "RANK": str(rank),
+                       "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank)})
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    import torch.distributed as dist
+    d = bench.Dist(backend="gloo")
+    cfg = W.CONFIGS["gdn"]
+    p = W.make_plan(cfg)
+    mine = list(range(rank, 4, world))               # requests of this rank
+    plan = oracle.Plan(cfg.d, cfg.d, cfg.heads, cfg.gate_kind, cfg.unit_kind, 0, p.bits, p.w)
+    pool = plan.new_pool(len(mine))
+    slots = np.arange(len(mine), dtype=np.int32)
+    plan.pack(pool, slots, W.initial_state(cfg, mine, heads=range(cfg.heads)))
+    si = W.step_inputs(cfg, 0, p, mine)
+    y, st = plan.decode_step(pool, slots, si.q, si.k, si.v, si.beta, si.gate)
+    out = [None] * world
+    dist.all_gather_object(out, {"reqs": mine, "y": y, "pool": pool, "st": st})
+    d.barrier()
+    m = d.max(float(rank + 1) * 1.5)
+    if rank == 0:
+        q.put((out, m))
+    d.close()
+
+
+@pytest.mark.timeout(300)
+def test_two_ranks_shard_requests_without_exchange():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    out, m = q.get(timeout=240)
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    assert m == 3.0                                  # max over ranks of (rank+1)*1.5
+    cfg = W.CONFIGS["gdn"]
+    p = W.make_plan(cfg)
+    plan = oracle.Plan(cfg.d, cfg.d, cfg.heads, cfg.gate_kind, cfg.unit_kind, 0, p.bits, p.w)
+    pool = plan.new_pool(4)
+    slots = np.arange(4, dtype=np.int32)
+    plan.pack(pool, slots, W.initial_state(cfg, range(4)))
+    si = W.step_inputs(cfg, 0, p, range(4))
+    y, st = plan.decode_step(pool, slots, si.q, si.k, si.v, si.beta, si.gate)
+    sb = plan.slot_bytes
+    for part in out:
+        assert part["st"] == 0
+        for a, r in enumerate(part["reqs"]):
+            assert np.array_equal(part["y"][a], y[r])
+            assert np.array_equal(part["pool"][a * sb:(a + 1) * sb], pool[r * sb:(r + 1) * sb])
