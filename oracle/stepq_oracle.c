@@ -44,7 +44,9 @@
  *   - the column-fit objective sum_i w_i^2 (X_ij - r_i c code_ij)^2 is
  *     evaluated in one stated binary32 order (see objective()), because the
  *     argmin it feeds is an integer decision that the CUDA kernels must
- *     reproduce exactly for multi-step rollouts to agree.
+ *     reproduce exactly for multi-step rollouts to agree; likewise the column
+ *     maximum max_i |X_ij / r_i| takes the quotient as |X_ij| times the
+ *     correctly rounded 1/r_i (times qmax_hi/qmax_i for rows of other widths).
  *
  * Parity status of each function is stated in its comment ("pinned by ...").
  */
@@ -429,6 +431,7 @@ int orc_quantize_head(const void *p, int h, const float *X, uint8_t *blob,
     float *kappa = (float *)calloc(dk, sizeof(float));
     int16_t *col = (int16_t *)calloc(dk, sizeof(int16_t));
     float *irho = (float *)calloc(dk, sizeof(float));
+    float *ikap = (float *)calloc(dk, sizeof(float));
     float *Aw = (float *)calloc(dk, sizeof(float));
     int qhi = 0;
 
@@ -489,6 +492,7 @@ int orc_quantize_head(const void *p, int h, const float *X, uint8_t *blob,
                 if (!active[i])
                     continue;
                 irho[i] = 1.0f / orc_half_to_float(rho[i]);
+                ikap[i] = irho[i] * kappa[i];
                 Aw[i] = (pl->w[h * dk + i] * orc_half_to_float(rho[i])) *
                         (pl->w[h * dk + i] * orc_half_to_float(rho[i]));
             }
@@ -499,7 +503,9 @@ int orc_quantize_head(const void *p, int h, const float *X, uint8_t *blob,
                     float z;
                     if (!active[i])
                         continue;
-                    z = (fabsf(X[i * dv + j]) / orc_half_to_float(rho[i])) * kappa[i];
+                    /* max_i |X_ij / r_i| (times kappa_i), the quotient taken as a
+                     * product with the correctly rounded 1/r_i, as in the objective */
+                    z = fabsf(X[i * dv + j]) * ikap[i];
                     if (z > M)
                         M = z;
                 }
@@ -530,7 +536,7 @@ int orc_quantize_head(const void *p, int h, const float *X, uint8_t *blob,
     }
     orc_pack_codes(p, h, codes, piv, rho, c, blob);
     free(codes); free(piv); free(rho); free(c); free(active); free(qmax); free(kappa); free(col);
-    free(irho); free(Aw);
+    free(irho); free(ikap); free(Aw);
     return status;
 }
 
