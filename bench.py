@@ -50,7 +50,27 @@ SMS, FP32_LANES = 148, 128
 METRIC = "quantized state-step throughput (head-updates/s) and HBM GB/s vs B200 peak"
 UNIT = "head-updates/s"
 ALU_OPS_PER_ENTRY = 60     # fp32 ops per quantised state entry in the fit + pack kernel
+ALU_OPS_PER_ENTRY_UNIFORM = 13  # the same without the column search (per-row scales only)
 PIVOT_OPS_PER_ENTRY = 6
+
+
+# quantiser variants: (fit mode, uniform width or None for the plan's widths,
+# FP16 pivots kept).  "spatial", "temporal" and "nopivot" are the ablations of
+# the method: the dual-axis fit alone on uniform widths, the lifetime-aware
+# widths alone with per-row scales, and the full method without pivots.
+MODES = {
+    "stepquant": (W.MODE_STEPQUANT, None, True),
+    "uniform8": (W.MODE_UNIFORM, 8, False),
+    "uniform6": (W.MODE_UNIFORM, 6, False),
+    "spatial": (W.MODE_STEPQUANT, 6, False),
+    "temporal": (W.MODE_UNIFORM, None, True),
+    "nopivot": (W.MODE_STEPQUANT, None, False),
+}
+
+
+def mode_plan(cfg, mode):
+    m, ub, piv = MODES[mode]
+    return m, W.make_plan(cfg, uniform_bits=ub, pivots=piv)
 
 
 def parse():
@@ -60,11 +80,19 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["stepq", "reference"], default="stepq")
     ap.add_argument("--config", choices=W.CONFIG_ORDER, default="gdn")
-    ap.add_argument("--mode", choices=["stepquant", "uniform8", "uniform6"], default="stepquant")
+    ap.add_argument("--mode", choices=list(MODES), default="stepquant")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--fp32-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="skip the CUDA-graph replay of the same steps")
+    ap.add_argument("--drift", action="store_true",
+                    help="instead of the throughput line: quantised rollouts vs the fp32 rollout")
+    ap.add_argument("--drift-arms", default="stepquant,uniform8,uniform6",
+                    help="comma-separated quantiser variants of the drift report")
+    ap.add_argument("--drift-steps", type=int, default=0,
+                    help="steps of the drift report (0: the workload's own step count)")
     ap.add_argument("--serial", action="store_true",
                     help="also time the step with both kernels on one stream, one layer")
     return ap.parse_args()
@@ -186,7 +214,7 @@ def readout_bytes(cfg, slot_bytes_per_head):
     return cfg.requests * (sum(slot_bytes_per_head) + cfg.heads * (qkv + 4 + gate + 4 * d))
 
 
-def fit_alu_ops(cfg, pin):
+def fit_alu_ops(cfg, pin, mode=W.MODE_STEPQUANT):
     d = cfg.d
     if cfg.unit_kind == W.UNIT_HEAD:
         q_rows = sum(d for b in pin.bits if b != 16)
@@ -194,7 +222,8 @@ def fit_alu_ops(cfg, pin):
     else:
         q_rows = int(np.sum(pin.bits != 16))
         p_rows = int(np.sum(pin.bits == 16))
-    return cfg.requests * d * (q_rows * ALU_OPS_PER_ENTRY + p_rows * PIVOT_OPS_PER_ENTRY)
+    per = ALU_OPS_PER_ENTRY if mode == W.MODE_STEPQUANT else ALU_OPS_PER_ENTRY_UNIFORM
+    return cfg.requests * d * (q_rows * per + p_rows * PIVOT_OPS_PER_ENTRY)
 
 
 class DeviceWorkload:
@@ -203,9 +232,7 @@ class DeviceWorkload:
 
         import quantized_delta_rule_decode_b200 as S
         self.S, self.cfg = S, cfg
-        ub = {"stepquant": None, "uniform8": 8, "uniform6": 6}[mode]
-        self.mode = W.MODE_UNIFORM if ub else W.MODE_STEPQUANT
-        self.pin = W.make_plan(cfg, uniform_bits=ub)
+        self.mode, self.pin = mode_plan(cfg, mode)
         d, H, R = cfg.d, cfg.heads, cfg.requests
         self.plan = S.stepq_plan_create(d, d, H, cfg.gate_kind, cfg.unit_kind, self.mode,
                                         self.pin.bits, self.pin.w)
@@ -346,6 +373,54 @@ def time_isolated(wl, steps, warmup):
     return rd, ft
 
 
+def time_graph(wl, steps):
+    """The same decode steps captured once into a CUDA graph and replayed.
+
+    One graph holds one period of the step sequence (every layer x every
+    input of the ring), both streams included; the pool views used in the
+    capture are fresh, so no step waits on an event recorded outside it."""
+    import torch
+    S, L = wl.S, wl.L
+    P = ctypes.c_void_p
+    period = wl.layers * 16 // math.gcd(wl.layers, 16)
+    cs, ss = torch.cuda.Stream(), torch.cuda.Stream()
+    pools = [S.stepq_pool_alloc(wl.plan, wl.nslots, p.buf) for p in wl.pools]
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    rcs = []
+    with torch.cuda.stream(cs):
+        g.capture_begin()
+        try:
+            for s in range(period):
+                a = list(wl.step_args[wl.args_index(s)])
+                a[1] = pools[s % wl.layers].handle
+                a[-2], a[-1] = P(cs.cuda_stream), P(ss.cuda_stream)
+                rcs.append(L.stepq_decode_step(*a))
+            cs.wait_stream(ss)
+        finally:
+            g.capture_end()
+    if any(rcs):
+        raise RuntimeError("decode step failed during graph capture: " + L.stepq_last_error().decode())
+    reps = max(1, steps // period)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(cs):
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a.record(cs)
+        for _ in range(reps):
+            g.replay()
+        b.record(cs)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / (reps * period)
+    del g
+    for p in pools:
+        S.stepq_pool_free(p)
+    cfg = wl.cfg
+    return {"ms_per_step": ms, "value": cfg.requests * cfg.heads / (ms * 1e-3), "unit": UNIT,
+            "steps_per_graph": period, "replays": reps, "kernel_nodes": 2 * period * reps}
+
+
 def time_serial(wl, steps, warmup):
     """Both kernels on one stream, one layer after another, no overlap."""
     import torch
@@ -460,10 +535,8 @@ class OracleRunner:
 
     def __init__(self, cfg, mode):
         import oracle
-        ub = {"stepquant": None, "uniform8": 8, "uniform6": 6}[mode]
-        m = W.MODE_UNIFORM if ub else W.MODE_STEPQUANT
+        m, self.pin = mode_plan(cfg, mode)
         self.cfg = cfg
-        self.pin = W.make_plan(cfg, uniform_bits=ub)
         self.plan = oracle.Plan(cfg.d, cfg.d, cfg.heads, cfg.gate_kind, cfg.unit_kind, m,
                                 self.pin.bits, self.pin.w)
         self.threads = os.cpu_count() or 1
@@ -493,6 +566,16 @@ class OracleRunner:
         for i in range(0, len(keys), len(self.keys)):
             list(self.ex.map(self._one, keys[i:i + len(self.keys)]))
 
+    def rate_single(self, seconds):
+        """One host thread, one (request, head) step after another."""
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < seconds:
+            self._one(self.keys[self.cursor % len(self.keys)])
+            self.cursor += 1
+            n += 1
+        return n / (time.perf_counter() - t0), n
+
     def rate(self, seconds):
         t0 = time.perf_counter()
         n = 0
@@ -500,6 +583,73 @@ class OracleRunner:
             self.run(self.threads)
             n += self.threads
         return n / (time.perf_counter() - t0), n
+
+
+def run_drift(args, dist):
+    """Quantised rollouts against the fp32 rollout of the same inputs.
+
+    From one packed S0, the chosen quantiser variants (by default the
+    workload's own plan with the STEPQuant fit, uniform INT8 and uniform
+    INT6) step side by side with the unquantised fp32 state, with fresh
+    seeded inputs every step.  At each
+    checkpoint: the relative Frobenius error of every (request, head) state
+    against the fp32 state, and the relative L2 error of y.  The pages report
+    accuracy only on real models, so these numbers are reported, not checked."""
+    import torch
+
+    import quantized_delta_rule_decode_b200 as S
+    cfg = W.CONFIGS[args.config]
+    steps = args.drift_steps or cfg.steps
+    d, H, R = cfg.d, cfg.heads, cfg.requests
+    slots = torch.from_numpy(W.slot_indices(cfg)).cuda()
+    pin = W.make_plan(cfg)
+    X0 = torch.from_numpy(W.initial_state(cfg)).cuda()
+    S32 = torch.zeros((cfg.pool_slots, H, d, d), dtype=torch.float32, device="cuda")
+    S32[slots.long()] = X0
+    arms = {}
+    for name in args.drift_arms.split(","):
+        mode, p = mode_plan(cfg, name)
+        plan = S.stepq_plan_create(d, d, H, cfg.gate_kind, cfg.unit_kind, mode, p.bits, p.w)
+        sb = S.stepq_plan_slot_bytes(plan)
+        buf = torch.zeros(cfg.pool_slots * sb, dtype=torch.uint8, device="cuda")
+        pool = S.stepq_pool_alloc(plan, cfg.pool_slots, buf)
+        S.stepq_pack(plan, pool, slots, X0)
+        arms[name] = {"plan": plan, "pool": pool, "slot_bytes": sb,
+                      "ws": torch.empty(S.stepq_workspace_bytes(plan, R), dtype=torch.uint8, device="cuda"),
+                      "y": torch.empty((R, H, d), dtype=torch.float32, device="cuda"), "points": []}
+    del X0
+    y32 = torch.empty((R, H, d), dtype=torch.float32, device="cuda")
+    Sq = torch.empty((R, H, d, d), dtype=torch.float32, device="cuda")
+    marks = sorted({m for m in (1, 16, 64, 256, 1024, 2048, 4096, steps) if m <= steps})
+    dt = torch.bfloat16 if cfg.bf16_inputs else torch.float32
+    t0 = time.perf_counter()
+    for step in range(steps):
+        si = W.step_inputs(cfg, step, pin)
+        q, k, v = (torch.from_numpy(a).to(dt).cuda() for a in (si.q, si.k, si.v))
+        beta, gate = torch.from_numpy(si.beta).cuda(), torch.from_numpy(si.gate).cuda()
+        S.stepq_fp32_step(S32, slots, q, k, v, beta, gate, y32, cfg.gate_kind)
+        for a in arms.values():
+            S.stepq_decode_step(a["plan"], a["pool"], slots, q, k, v, beta, gate, a["y"], a["ws"])
+        if step + 1 in marks:
+            ref = S32[slots.long()]
+            rn = ref.flatten(2).norm(dim=2)
+            for name, a in arms.items():
+                S.stepq_unpack(a["plan"], a["pool"], slots, Sq)
+                e = (Sq - ref).flatten(2).norm(dim=2) / rn
+                ey = float((a["y"] - y32).norm() / y32.norm())
+                a["points"].append({"step": step + 1, "state_rel_fro_mean": float(e.mean()),
+                                    "state_rel_fro_median": float(e.median()),
+                                    "state_rel_fro_max": float(e.max()), "y_rel_l2": ey})
+    torch.cuda.synchronize()
+    status = {n: S.stepq_get_status(a["pool"]) for n, a in arms.items()}
+    out = {"report": "rollout drift of quantised states vs the fp32 state", "config": args.config,
+           "workload": workload_config(cfg, "stepquant", None)["workload"], "steps": steps,
+           "data": "synthetic (seeded; workload.py)", "seconds": time.perf_counter() - t0,
+           "arms": {n: {"slot_bytes": a["slot_bytes"],
+                        "compression_vs_fp32": H * d * d * 4 / a["slot_bytes"],
+                        "device_status": status[n], "points": a["points"]} for n, a in arms.items()}}
+    if dist.rank == 0:
+        print(json.dumps(out), flush=True)
 
 
 def cpu_model():
@@ -544,7 +694,7 @@ def run_reference(args, dist):
 
 
 def workload_config(cfg, mode, wl):
-    pin = wl.pin if wl is not None else W.make_plan(cfg)
+    pin = wl.pin if wl is not None else mode_plan(cfg, mode)[1]
     counts = {int(b): int(np.sum(pin.bits == b)) for b in (4, 6, 8, 16) if np.sum(pin.bits == b)}
     c = {"workload": f"{cfg.name}: {cfg.requests} requests x {cfg.heads} heads, d_k=d_v={cfg.d}, "
                      f"{'KDA per-key-row' if cfg.gate_kind else 'GDN scalar'} gates, "
@@ -590,6 +740,12 @@ def main():
         run_reference(args, dist)
         dist.close()
         return
+    if args.drift:
+        import torch
+        torch.cuda.set_device(dist.local)
+        run_drift(args, dist)
+        dist.close()
+        return
     import torch
     torch.cuda.set_device(dist.local)
     peaks = {}
@@ -618,7 +774,7 @@ def main():
 
     rd_bytes = readout_bytes(cfg, wl.head_bytes)
     rd_gbs = rd_bytes / (readout_ms * 1e-3) / 1e9
-    ops = fit_alu_ops(cfg, wl.pin)
+    ops = fit_alu_ops(cfg, wl.pin, wl.mode)
     clk_mhz = float(peaks.get("sm_max_mhz", 1965.0))
     alu_peak = SMS * FP32_LANES * clk_mhz * 1e6 / 1e12   # T fp32 lane-ops/s
     fit_tops = ops / (fit_ms * 1e-3) / 1e12
@@ -650,6 +806,11 @@ def main():
     e2e_ms, h2d, d2h = time_e2e(wl, args.e2e_steps, max(3, args.warmup // 5))
     e2e_ms = dist.max(e2e_ms)
     e2e_value = hu / (e2e_ms / args.e2e_steps * 1e-3)
+    graph = time_graph(wl, args.steps) if args.graph else None
+    graph_dev = dist.max(graph["ms_per_step"]) if graph else None
+    if graph:
+        graph["ms_per_step"] = graph_dev
+        graph["value"] = dist.world * cfg.requests * cfg.heads / (graph_dev * 1e-3)
     fp32 = time_fp32(cfg, wl.pin, args.fp32_steps, 10)
     if fp32 is not None:
         fp32["frac_hbm"] = fp32["hbm_gbs"] / hbm_peak
@@ -659,7 +820,9 @@ def main():
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
         orc = OracleRunner(cfg, args.mode)
         rate, n = orc.rate(args.cpu_seconds)
+        rate1, n1 = orc.rate_single(max(2.0, args.cpu_seconds / 4))
         cpu = {"value": rate, "unit": UNIT, "cores": orc.threads, "kind": "oracle",
+               "value_1thread": rate1,
                "sample": f"{n} (request, head) oracle steps of the {cfg.name} workload "
                          f"({orc.R} requests x {cfg.heads} heads cycled) in {args.cpu_seconds:.0f} s",
                "cpu": cpu_model()}
@@ -675,6 +838,7 @@ def main():
                 "roofline": roof, "kernels": kern,
                 "fp32_state_baseline": fp32,
                 "serial_step": serial,
+                "graph": graph,
                 "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps,

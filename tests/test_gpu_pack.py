@@ -26,6 +26,11 @@ CASES = [
     ("rollout", W.MODE_UNIFORM, 8, 2),
     ("rollout", W.MODE_UNIFORM, 6, 2),
     ("gdn", W.MODE_STEPQUANT, 4, 2),     # every head 4-bit: the search moves most
+    # ablations: lifetime-aware widths with per-row scales only (temporal),
+    # the dual-axis fit on uniform widths of key rows (spatial)
+    ("gdn", W.MODE_UNIFORM, None, 2),
+    ("kda", W.MODE_UNIFORM, None, 2),
+    ("kda", W.MODE_STEPQUANT, 6, 2),
 ]
 
 

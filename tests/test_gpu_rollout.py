@@ -8,7 +8,8 @@ dequantised state's relative Frobenius drift from the oracle's stays
 runs in full on the GPU, in the launch configuration bench.py times, and is
 compared on a fixed subset of 2 requests x 16 heads.  Since the kernels
 evaluate delta, X and the column objective in the oracle's order, the
-rollouts stay identical, and the tests also check the packed bytes.
+rollouts stay identical, and the tests also check the packed bytes (every step for the
+short rollouts).
 """
 
 from concurrent.futures import ThreadPoolExecutor
@@ -23,7 +24,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _rollout(name, steps, compare_reqs, gpu_reqs, mode=W.MODE_STEPQUANT, ub=None, every=32,
-             exact=True):
+             bytes_every=None):
     import torch
     cfg = W.CONFIGS[name]
     pair = Pair(cfg, mode=mode, uniform_bits=ub)
@@ -61,6 +62,13 @@ def _rollout(name, steps, compare_reqs, gpu_reqs, mode=W.MODE_STEPQUANT, ub=None
             yo[key] = yy
 
         list(ex.map(one, keys))
+        if bytes_every and (step % bytes_every == bytes_every - 1 or step == steps - 1):
+            # the packed slots, byte for byte: a transient divergence (one row
+            # factor off by a half ulp for one step) cannot pass unseen
+            gb = pool_to_host(pool)
+            for r in compare_reqs:
+                a, b = r * pair.slot_bytes, (r + 1) * pair.slot_bytes
+                assert np.array_equal(gb[a:b], o[a:b]), f"step {step}: request {r} state differs"
         if step % every == every - 1 or step == steps - 1:
             S.stepq_unpack(pair.gpu, pool, sl, Sg)
             torch.cuda.synchronize()
@@ -69,11 +77,6 @@ def _rollout(name, steps, compare_reqs, gpu_reqs, mode=W.MODE_STEPQUANT, ub=None
             for r in compare_reqs:
                 d = rel_l2(gS[r], oS[r])
                 worst_drift = max(worst_drift, d)
-            if exact:
-                gb = pool_to_host(pool)
-                for r in compare_reqs:
-                    a, b = r * pair.slot_bytes, (r + 1) * pair.slot_bytes
-                    assert np.array_equal(gb[a:b], o[a:b]), f"step {step}: request {r} state differs"
             yg = y.cpu().numpy()
             worst_y = max(worst_y, max(rel_l2(yg[r, h], yo[(r, h)]) for (r, h) in keys))
     ex.shutdown()
@@ -82,23 +85,23 @@ def _rollout(name, steps, compare_reqs, gpu_reqs, mode=W.MODE_STEPQUANT, ub=None
 
 
 def test_rollout_tiny_256_steps():
-    drift, ydiff = _rollout("tiny", 256, [0], 1, every=8)
+    drift, ydiff = _rollout("tiny", 256, [0], 1, every=8, bytes_every=1)
     assert drift <= 1e-3, drift
 
 
 def test_rollout_tiny_uniform8_256_steps():
-    drift, _ = _rollout("tiny", 256, [0], 1, mode=W.MODE_UNIFORM, ub=8, every=16)
+    drift, _ = _rollout("tiny", 256, [0], 1, mode=W.MODE_UNIFORM, ub=8, every=16, bytes_every=1)
     assert drift <= 1e-3, drift
 
 
 def test_rollout_kda_256_steps():
     """Per-key-row gates and widths (with FP16 pivot rows), 2 requests."""
-    drift, _ = _rollout("kda", 256, [0, 1], 2, every=64)
+    drift, _ = _rollout("kda", 256, [0, 1], 2, every=64, bytes_every=1)
     assert drift <= 1e-3, drift
 
 
 @pytest.mark.slow
 def test_rollout_long_4096_steps_subset():
     """128 requests x 16 heads on the GPU for 4096 steps; 2 x 16 compared."""
-    drift, _ = _rollout("rollout", 4096, [0, 1], 128, every=256)
+    drift, _ = _rollout("rollout", 4096, [0, 1], 128, every=256, bytes_every=256)
     assert drift <= 1e-3, drift

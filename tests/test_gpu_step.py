@@ -115,6 +115,16 @@ def test_step_rollout_uniform8_single_stream():
     _run_case("rollout", mode=W.MODE_UNIFORM, ub=8, R=3, two_streams=False)
 
 
+def test_step_kda_temporal_only():
+    """Ablation: per-key-row widths and pivots, per-row scales only (no column fit)."""
+    _run_case("kda", mode=W.MODE_UNIFORM, R=2, steps=2)
+
+
+def test_step_kda_spatial_only():
+    """Ablation: the dual-axis fit on uniform 6-bit key rows, no pivots."""
+    _run_case("kda", mode=W.MODE_STEPQUANT, ub=6, R=2, steps=2)
+
+
 def test_two_streams_equal_one_stream_and_split_calls():
     """decode_step on two streams == on one stream == readout + fitpack called separately."""
     import torch
