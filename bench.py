@@ -65,11 +65,58 @@ MODES = {
     "spatial": (W.MODE_STEPQUANT, 6, False),
     "temporal": (W.MODE_UNIFORM, None, True),
     "nopivot": (W.MODE_STEPQUANT, None, False),
+    "calibrated": (W.MODE_STEPQUANT, None, True),   # widths from calibrated_plan()
 }
+
+CAL_STEPS, CAL_SNAPSHOTS, CAL_REQUESTS = 64, 4, 16
+CAL_STEP_BASE = 1 << 24     # calibration inputs: step indices no decode run uses
+
+
+def calibrated_plan(cfg):
+    """The workload's plan with widths and pivots from the lifetime-aware
+    allocation, calibrated on fp32 rollouts of held-out requests and steps.
+
+    Calibration states: CAL_REQUESTS requests numbered after the workload's
+    own, stepped CAL_STEPS times by the fp32 kernel from their seeded S0 with
+    seeded inputs of step indices CAL_STEP_BASE + t, snapshotted CAL_SNAPSHOTS
+    times; lifetimes from the plan's gates; the budget and the pivot count of
+    the workload's own recipe."""
+    import torch
+
+    import quantized_delta_rule_decode_b200 as S
+    from quantized_delta_rule_decode_b200 import calibrate
+    pin = W.make_plan(cfg)
+    d, H = cfg.d, cfg.heads
+    reqs = list(range(cfg.requests, cfg.requests + CAL_REQUESTS))
+    Sx = torch.from_numpy(W.initial_state(cfg, reqs)).cuda()
+    slots = torch.arange(len(reqs), dtype=torch.int32, device="cuda")
+    dt = torch.bfloat16 if cfg.bf16_inputs else torch.float32
+    y = torch.empty((len(reqs), H, d), dtype=torch.float32, device="cuda")
+    states = []
+    every = CAL_STEPS // CAL_SNAPSHOTS
+    for t in range(CAL_STEPS):
+        si = W.step_inputs(cfg, CAL_STEP_BASE + t, pin, reqs)
+        q, k, v = (torch.from_numpy(a).to(dt).cuda() for a in (si.q, si.k, si.v))
+        beta, gate = torch.from_numpy(si.beta).cuda(), torch.from_numpy(si.gate).cuda()
+        S.stepq_fp32_step(Sx, slots, q, k, v, beta, gate, y, cfg.gate_kind)
+        if (t + 1) % every == 0:
+            states.append(Sx.clone())
+    g = np.asarray(pin.gate, np.float32)
+    if cfg.unit_kind == W.UNIT_ROW:
+        g = g.reshape(-1) if cfg.gate_kind == W.GATE_DIAG else np.repeat(g, d)
+    elif g.ndim == 2:
+        g = None
+    gates = g[None, :, None] if g is not None else np.asarray(pin.gate, np.float32)[None]
+    n_piv = int(np.sum(pin.bits == 16))
+    bits, _, _ = calibrate.calibrate_bits(d, d, H, cfg.gate_kind, cfg.unit_kind, pin.w, states, gates,
+                                          cfg.budget, n_piv)
+    return W.PlanInputs(bits=bits, w=pin.w, half_life=pin.half_life, gate=pin.gate)
 
 
 def mode_plan(cfg, mode):
     m, ub, piv = MODES[mode]
+    if mode == "calibrated":
+        return m, calibrated_plan(cfg)
     return m, W.make_plan(cfg, uniform_bits=ub, pivots=piv)
 
 
@@ -85,11 +132,13 @@ def parse():
     ap.add_argument("--fp32-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--isolated-steps", type=int, default=500,
+                    help="steps of the per-kernel timing with each kernel alone")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="skip the CUDA-graph replay of the same steps")
     ap.add_argument("--drift", action="store_true",
                     help="instead of the throughput line: quantised rollouts vs the fp32 rollout")
-    ap.add_argument("--drift-arms", default="stepquant,uniform8,uniform6",
+    ap.add_argument("--drift-arms", default="stepquant,calibrated,uniform8,uniform6",
                     help="comma-separated quantiser variants of the drift report")
     ap.add_argument("--drift-steps", type=int, default=0,
                     help="steps of the drift report (0: the workload's own step count)")
@@ -714,10 +763,10 @@ def workload_config(cfg, mode, wl):
 
 
 def src_sha():
+    """Hash of the sources that define the device kernels (not the host API)."""
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.join(ROOT, "quantized_delta_rule_decode_b200", "csrc"))):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(ROOT, "quantized_delta_rule_decode_b200", "csrc", f), "rb").read())
+    for f in ("stepq_kernels.cu", "stepq_internal.cuh"):
+        h.update(open(os.path.join(ROOT, "quantized_delta_rule_decode_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -765,7 +814,7 @@ def main():
     ms, readout_ms, fit_ms, clocks = time_device(wl, args.steps, args.warmup, dist, gpu_index)
     # which kernel bounds the step: each kernel timed alone (the overlapped
     # durations above share the SMs with the other stream)
-    iso_readout_ms, iso_fit_ms = time_isolated(wl, 500, args.warmup)
+    iso_readout_ms, iso_fit_ms = time_isolated(wl, args.isolated_steps, args.warmup)
     ms_step = ms / args.steps
     hu = dist.world * cfg.requests * cfg.heads
     value = hu / (ms_step * 1e-3)
@@ -787,8 +836,8 @@ def main():
                         "us_alone": iso_fit_ms * 1e3, "tops_alone": iso_fit_tops,
                         "frac_alu_alone": iso_fit_tops / alu_peak},
             "note": "us: average launch duration inside the timed region, where the two streams overlap "
-                    "and share the SMs; us_alone: the kernel alone on one stream (500 steps after the "
-                    "timed region); the roofline kernel is the one with the longer us_alone"}
+                    f"and share the SMs; us_alone: the kernel alone on one stream ({args.isolated_steps} steps "
+                    "after the timed region); the roofline kernel is the one with the longer us_alone"}
     if iso_fit_ms >= iso_readout_ms:
         roof = {"kernel": "fitpack (k_quant, fit+pack)", "bound": "alu", "achieved": fit_tops,
                 "peak": alu_peak, "unit": "T fp32 lane-ops/s", "frac": fit_tops / alu_peak,

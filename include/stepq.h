@@ -78,7 +78,7 @@ extern "C" {
  * calibrated row-impact weights (hyper.ai summary, "Method": row-impact score
  * per key row).
  *
- *   d_k, d_v   state shape per head; this build runs d_k == d_v in {64, 128}
+ *   d_k, d_v   state shape per head; the library runs d_k == d_v in {64, 128}
  *              (others: STEPQ_ERR_UNSUPPORTED).
  *   n_heads    heads per layer, >= 1.
  *   gate_kind  STEPQ_GATE_SCALAR or STEPQ_GATE_DIAG.
@@ -107,7 +107,7 @@ typedef struct stepq_pool stepq_pool;
  * Create a plan: validates the description, computes the packed byte layout
  * of one slot and uploads the per-head / per-row tables to the current device.
  *
- * Layout of one slot (the pages give no byte format; this is the build's):
+ * Layout of one slot (the pages give no byte format; this one is the library's own):
  * the heads' blobs in head order, each starting on a 16-byte boundary; the
  * slot stride is their total rounded up to 256 bytes.  A head blob is its key
  * rows in ascending order -- a b-bit row holds d_v codes stored as
@@ -279,6 +279,62 @@ STEPQ_API int stepq_decode_step_static(const stepq_plan *plan, stepq_pool *pool,
                                        const void *q, const void *k, const void *v,
                                        const float *beta, const float *gate, float *y,
                                        void *main_stream, void *side_stream);
+
+/* ------------------------------------------------------------------------
+ * Offline calibration: lifetime-aware bit allocation.  hyper.ai summary,
+ * section "Method" (the Lifetime-Aware Bit Allocation paragraph); rcap.io
+ * post, "Temporal" part: before decoding, each state unit (a head, or one key
+ * row) gets a width from {4, 6, 8} bits, or FP16 as a pivot, from its
+ * reconstruction distortion at each width and its memory lifetime, under an
+ * average bit budget.  The three calls below are the measurement, the
+ * lifetime weight and the selection; a calibration run strings them together
+ * (quantise calibration states with a plan of one width per call to
+ * stepq_pack, measure, repeat for each width, then select).
+ * ------------------------------------------------------------------------ */
+
+/* Per-unit squared reconstruction error of packed slots against the states
+ * they were packed from: dist[r][u] = sum over unit u's entries of
+ * (X[r] - S[r])^2, S the state reconstructed from the slot slot_idx[r], each
+ * difference and square in double.  Units follow the plan: one per head
+ * (unit_kind HEAD, dist is [n][n_heads]) or one per key row (unit_kind ROW,
+ * [n][n_heads * d_k], row i of head h at h * d_k + i).
+ *   X     device, fp32 [n][n_heads][d_k][d_v] (caller-owned, read only)
+ *   dist  device, float64 [n][units] (caller-owned, written)
+ * Asynchronous on `stream`.  A slot index outside the pool sets
+ * STEPQ_DEV_BAD_SLOT and leaves that request's entries of dist unwritten.
+ * The summation order inside a unit is the kernel's own (a tree over
+ * columns, then rows in ascending order). */
+STEPQ_API int stepq_unit_distortion(const stepq_plan *plan, stepq_pool *pool,
+                                    const int32_t *slot_idx, int64_t n, const float *X,
+                                    double *dist, void *stream);
+
+/* Lifetime weight of each unit from its retention gates over calibration
+ * steps: ell_u = mean of log(g) over the unit's gates and the steps, the error
+ * left after j updates is exp(j ell_u), and the weight is
+ * sum_{j >= 0} exp(j ell_u) = 1 / (1 - exp(ell_u)).
+ *   gate    host, fp32 [n_steps][n_units][gates_per_unit], every value in (0, 1)
+ *   weight  host, float64 [n_units]
+ * Host-only (no device work).  STEPQ_ERR_INVALID if a gate is outside (0, 1)
+ * or a size is not positive; nothing is written then. */
+STEPQ_API int stepq_lifetime_weight(int64_t n_units, int64_t n_steps, int32_t gates_per_unit,
+                                    const float *gate, double *weight);
+
+/* Widths minimising the lifetime-weighted distortion under an average budget.
+ *   weight  host, float64 [n_units] (stepq_lifetime_weight), > 0 and finite
+ *   dist    host, float64 [n_units][3]: distortion at 4, 6, 8 bits, >= 0, finite
+ *   budget_bits  4, 6 or 8: the average width of the non-pivot units may not
+ *           exceed it
+ *   n_pivots  units kept in FP16: those of largest risk weight * dist(budget
+ *           width), ties to the lower unit index
+ *   bits    host, uint8 [n_units]: 4, 6, 8, or 16 for a pivot (written)
+ * The other units' widths are the exact minimum of sum weight_u * dist_u(b_u)
+ * subject to sum b_u <= budget_bits * (n_units - n_pivots), taken by a
+ * recurrence over units in ascending order with the number of 2-bit upgrades
+ * left as its state; on equal sums the earlier unit takes the smaller width.
+ * Host-only; memory O(n_units^2) bytes for budget 6 (16.8 MB at 4096 units).
+ * STEPQ_ERR_INVALID on bad arguments (nothing written). */
+STEPQ_API int stepq_allocate_bits(int64_t n_units, const double *weight, const double *dist,
+                                  int32_t budget_bits, int64_t n_pivots, uint8_t *bits);
 
 /* Synchronously read the pool's device status word (STEPQ_DEV_* bits, OR-ed
  * over every call since the last clear).  Waits for the device to go idle. */

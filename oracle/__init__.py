@@ -67,6 +67,8 @@ def lib():
         L.orc_fp32_step_head.argtypes = [I, I, P, P, P, P, F, P, I, P]
         L.orc_fp32_step.argtypes = [I, I, I, I, P, I64, P, I64, P, P, P, P, P, P]
         L.orc_fp32_step.restype = I
+        L.orc_unit_distortion.argtypes = [P, P, I64, P, I64, P, P]
+        L.orc_unit_distortion.restype = I
         _lib = L
     return _lib
 
@@ -187,6 +189,15 @@ class Plan:
         S = np.zeros((sl.size, self.H, self.dk, self.dv), np.float32)
         st = lib().orc_unpack(self.h, _p(pool), pool.size // self.slot_bytes, _p(sl), sl.size, _p(S))
         return S, st
+
+    def unit_distortion(self, pool, slot_idx, X):
+        """Per-unit squared reconstruction error [n][units] (float64) and status."""
+        sl = np.ascontiguousarray(slot_idx, np.int32)
+        units = self.H * self.dk if self.unit_kind else self.H
+        dist = np.zeros((sl.size, units), np.float64)
+        st = lib().orc_unit_distortion(self.h, _p(pool), pool.size // self.slot_bytes, _p(sl), sl.size,
+                                       _p(_f32(X)), _p(dist))
+        return dist, st
 
     def decode_step(self, pool, slot_idx, q, k, v, beta, gate):
         sl = np.ascontiguousarray(slot_idx, np.int32)

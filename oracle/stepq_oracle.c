@@ -26,10 +26,10 @@
  *        least squares with squared impact weights, quantise X/(r c)).
  *   The deterministic column fit (8 candidates alpha * max_i|X_ij/r_i| / qmax,
  *   alpha = 1.0 .. 0.65, ties to the larger alpha), the round-half-even codes
- *   and the per-unit widths {4,6,8} are the benchmark spec's concrete form of
- *   [P3]'s `fit_weighted_lsq` and `quantize`.
+ *   and the per-unit widths {4,6,8} are the concrete form taken here of
+ *   [P3]'s `fit_weighted_lsq` and `quantize`, which the pages leave open.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *   - row magnitude = max_j |X_ij|; objective weight = w_i^2 (w as given).
  *   - per-row widths inside one head (key-row units): the row factor absorbs
  *     the width, rho_i = r_i * qmax_hi / qmax_i, so each row's codes span its
@@ -656,6 +656,57 @@ int orc_decode_step(const void *p, uint8_t *pool, int64_t num_slots, const int32
                                 q + rh * d, k + rh * d, v + rh * dv, beta[rh], g, y + rh * dv, NULL);
         }
     }
+    return st;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Per-unit reconstruction distortion, the input of the lifetime-aware bit   */
+/* allocation ([P1], section "Method": the distortion of every state unit    */
+/* at each candidate width is measured on calibration states).               */
+/*   D_u = sum over the unit's entries of (X_ij - S_ij)^2,                   */
+/* S the dequantised packed state; each difference taken in double from the  */
+/* binary32 values, squares summed in double over rows then columns, in      */
+/* ascending order.  A unit is a head (unit_kind 0) or one key row           */
+/* (unit_kind 1); dist is [n][units], units = H or H*dk.  Rows of slots out  */
+/* of range are skipped (status BAD_SLOT, their entries left untouched).     */
+/* Pinned by tests/test_oracle_alloc.py: zero for states that the quantiser  */
+/* represents exactly, and equal to the squared Frobenius error of          */
+/* orc_unpack's reconstruction computed independently.                       */
+/* ------------------------------------------------------------------------ */
+
+int orc_unit_distortion(const void *p, const uint8_t *pool, int64_t num_slots,
+                        const int32_t *slot_idx, int64_t n, const float *X, double *dist)
+{
+    const orc_plan *pl = (const orc_plan *)p;
+    int dk = pl->dk, dv = pl->dv, H = pl->H, h, i, j, st = 0;
+    int64_t r;
+    size_t hs = (size_t)dk * dv;
+    size_t units = pl->unit_kind ? (size_t)H * dk : (size_t)H;
+    float *S = (float *)malloc(sizeof(float) * hs);
+    for (r = 0; r < n; r++) {
+        if (slot_idx[r] < 0 || slot_idx[r] >= num_slots) {
+            st |= ORC_STATUS_BAD_SLOT;
+            continue;
+        }
+        for (h = 0; h < H; h++) {
+            const float *Xh = X + ((size_t)r * H + h) * hs;
+            double head = 0.0;
+            orc_dequantize_head(p, h, pool + (size_t)slot_idx[r] * pl->slot_bytes + pl->head_off[h], S);
+            for (i = 0; i < dk; i++) {
+                double row = 0.0;
+                for (j = 0; j < dv; j++) {
+                    double e = (double)Xh[i * dv + j] - (double)S[i * dv + j];
+                    row += e * e;
+                }
+                if (pl->unit_kind)
+                    dist[(size_t)r * units + (size_t)h * dk + i] = row;
+                head += row;
+            }
+            if (!pl->unit_kind)
+                dist[(size_t)r * units + h] = head;
+        }
+    }
+    free(S);
     return st;
 }
 

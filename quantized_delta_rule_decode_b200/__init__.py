@@ -25,6 +25,7 @@ from ._ffi import (  # noqa: F401
     StepqError,
     library_path,
     load_library,
+    stepq_allocate_bits,
     stepq_clear_status,
     stepq_decode_fitpack,
     stepq_decode_readout,
@@ -34,10 +35,12 @@ from ._ffi import (  # noqa: F401
     stepq_fp32_step,
     stepq_get_status,
     stepq_host_workspace_bytes,
+    stepq_lifetime_weight,
     stepq_pack,
     stepq_plan_create,
     stepq_plan_destroy,
     stepq_plan_head_layout,
+    stepq_unit_distortion,
     stepq_plan_slot_bytes,
     stepq_pool_alloc,
     stepq_pool_free,

@@ -37,6 +37,9 @@ _SIGS = {
     "stepq_host_workspace_bytes": [_P, _I64, _I32, ctypes.POINTER(_SZ)],
     "stepq_decode_step_host": [_P, _P, _P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P],
     "stepq_decode_step_static": [_P, _P, _P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P, _P],
+    "stepq_unit_distortion": [_P, _P, _P, _I64, _P, _P, _P],
+    "stepq_lifetime_weight": [_I64, _I64, _I32, _P, _P],
+    "stepq_allocate_bits": [_I64, _P, _P, _I32, _I64, _P],
     "stepq_get_status": [_P, ctypes.POINTER(ctypes.c_uint32)],
     "stepq_clear_status": [_P, _P],
     "stepq_last_error": [],
@@ -289,6 +292,41 @@ def stepq_fp32_step(S, slot_idx, q, k, v, beta, gate, y, gate_kind, dev_status=N
           num_slots, s, n, _ptr(q, q.dtype, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"),
           _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
           _ptr(y, torch.float32, "y"), _ptr(dev_status, name="dev_status"), _stream(stream))
+
+
+def stepq_unit_distortion(plan: Plan, pool: Pool, slot_idx, X, dist=None, stream=None):
+    """Per-unit squared reconstruction error [n][units] (float64, on the device)."""
+    import torch
+    s, n = _slots(slot_idx)
+    units = plan.n_heads * plan.d_k if plan.unit_kind == UNIT_ROW else plan.n_heads
+    if dist is None:
+        dist = torch.empty((n, units), dtype=torch.float64, device=X.device)
+    _call("stepq_unit_distortion", plan.handle, pool.handle, s, n, _ptr(X, torch.float32, "X"),
+          _ptr(dist, torch.float64, "dist"), _stream(stream))
+    return dist
+
+
+def stepq_lifetime_weight(gate) -> np.ndarray:
+    """gate: host float32 [n_steps][n_units][gates_per_unit] (or [n_steps][n_units])."""
+    g = np.ascontiguousarray(gate, np.float32)
+    if g.ndim == 2:
+        g = g[:, :, None]
+    steps, units, per = g.shape
+    out = np.zeros(units, np.float64)
+    _call("stepq_lifetime_weight", units, steps, per, g.ctypes.data_as(_P), out.ctypes.data_as(_P))
+    return out
+
+
+def stepq_allocate_bits(weight, dist, budget_bits: int, n_pivots: int) -> np.ndarray:
+    """weight [n_units] float64, dist [n_units][3] float64 (4, 6, 8 bits) -> uint8 widths."""
+    w = np.ascontiguousarray(weight, np.float64)
+    d = np.ascontiguousarray(dist, np.float64)
+    if d.shape != (w.size, 3):
+        raise ValueError("dist must be [n_units][3]")
+    bits = np.zeros(w.size, np.uint8)
+    _call("stepq_allocate_bits", w.size, w.ctypes.data_as(_P), d.ctypes.data_as(_P), int(budget_bits),
+          int(n_pivots), bits.ctypes.data_as(_P))
+    return bits
 
 
 def stepq_get_status(pool: Pool) -> int:

@@ -146,7 +146,7 @@ int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out) {
         if (!(d.w[i] > 0.0f) || isinf(d.w[i]))
             return fail(STEPQ_ERR_INVALID, "w[%zu] must be finite and > 0", i);
     if (dk != dv || (dk != 64 && dk != 128))
-        return fail(STEPQ_ERR_UNSUPPORTED, "this build runs d_k == d_v in {64, 128} (got %d x %d)", dk, dv);
+        return fail(STEPQ_ERR_UNSUPPORTED, "the library runs d_k == d_v in {64, 128} (got %d x %d)", dk, dv);
 
     stepq_plan *p = new stepq_plan();
     p->dk = dk; p->dv = dv; p->H = H;
@@ -360,6 +360,23 @@ int stepq_unpack(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_i
     return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "unpack launch");
 }
 
+int stepq_unit_distortion(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_idx,
+                          int64_t n, const float *X, double *dist, void *stream) {
+    g_err.clear();
+    int rc = check_pool(plan, pool);
+    if (!rc) rc = check_rows(plan, slot_idx, n);
+    if (rc) return rc;
+    if (n == 0) return STEPQ_OK;
+    if ((rc = check_inputs(X, "X")) || (rc = check_inputs(dist, "dist"))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((rc = wait_pending_fit(pool, s))) return rc;
+    stepq::StepArgs a = base_args(plan, pool, slot_idx, n);
+    a.X = X;
+    a.dist = dist;
+    cudaError_t e = stepq::launch_distortion(plan->dev, a, s);
+    return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "distortion launch");
+}
+
 static int check_step_inputs(const stepq_plan *plan, int64_t n, int32_t qkv_dtype, const void *q,
                              const void *k, const void *v, const float *beta, const float *gate,
                              const float *y, const void *ws, size_t ws_bytes, bool readout) {
@@ -516,7 +533,7 @@ int stepq_fp32_step(int32_t d_k, int32_t d_v, int32_t n_heads, int32_t gate_kind
                     const float *gate, float *y, uint32_t *dev_status, void *stream) {
     g_err.clear();
     if (d_k != d_v || (d_k != 64 && d_k != 128))
-        return fail(STEPQ_ERR_UNSUPPORTED, "this build runs d_k == d_v in {64, 128}");
+        return fail(STEPQ_ERR_UNSUPPORTED, "the library runs d_k == d_v in {64, 128}");
     if (n_heads <= 0 || num_slots <= 0) return fail(STEPQ_ERR_INVALID, "n_heads, num_slots must be positive");
     if (gate_kind != STEPQ_GATE_SCALAR && gate_kind != STEPQ_GATE_DIAG)
         return fail(STEPQ_ERR_INVALID, "gate_kind %d unknown", gate_kind);

@@ -51,6 +51,7 @@ struct StepArgs {
     float *delta;      // workspace [n][H][dv]
     const float *X;    // pack input [n][H][dk][dv]
     float *S_out;      // unpack output
+    double *dist;      // per-unit distortion output [n][units]
     uint32_t *status;
 };
 
@@ -59,6 +60,7 @@ cudaError_t launch_readout(const PlanDev &P, const StepArgs &a, int qkv_dtype, c
 cudaError_t launch_fitpack(const PlanDev &P, const StepArgs &a, int qkv_dtype, cudaStream_t s);
 cudaError_t launch_pack(const PlanDev &P, const StepArgs &a, cudaStream_t s);
 cudaError_t launch_unpack(const PlanDev &P, const StepArgs &a, cudaStream_t s);
+cudaError_t launch_distortion(const PlanDev &P, const StepArgs &a, cudaStream_t s);
 cudaError_t launch_fp32_step(int d, int H, int gate_kind, int qkv_dtype, float *S, int64_t num_slots,
                              const int32_t *slot_idx, int64_t n, const void *q, const void *k,
                              const void *v, const float *beta, const float *gate, float *y,

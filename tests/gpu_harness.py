@@ -4,7 +4,7 @@ The GPU side is driven only through the C ABI (``quantized_delta_rule_decode_b20
 ctypes over libstepq.so); the expected values come only from ``oracle/``;
 both read their inputs from ``workload`` (seeded, synthetic).
 
-Comparison rules (derived in DESIGN.md, "Parity contract"):
+Comparison rules:
 
 * packing from an identical X is bit-exact, except that the column-scale
   argmin may pick another candidate when the two candidates' objectives are

@@ -1,10 +1,9 @@
 """Multi-step rollouts, GPU vs oracle, each side evolving its own state.
 
 Both start from the same packed state (packed by the oracle) and take the
-same seeded inputs every step (fresh q, k, v, beta per step).  The contract
-(task statement, restated in the design doc): over a 256-step rollout the
-dequantised state's relative Frobenius drift from the oracle's stays
-<= 1e-3.  The long rollout workload (128 requests x 16 heads, 4096 steps)
+same seeded inputs every step (fresh q, k, v, beta per step).  The contract:
+over a 256-step rollout the dequantised state's relative Frobenius drift
+from the oracle's stays <= 1e-3.  The long rollout workload (128 requests x 16 heads, 4096 steps)
 runs in full on the GPU, in the launch configuration bench.py times, and is
 compared on a fixed subset of 2 requests x 16 heads.  Since the kernels
 evaluate delta, X and the column objective in the oracle's order, the

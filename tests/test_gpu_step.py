@@ -5,11 +5,11 @@ y = X^T q (before requantising) -> refit scales -> pack back (rcap.io post,
 decode-step pseudocode; hyper.ai summary, "Method").  Both sides start from
 the same packed state (packed by the oracle, copied to the device).
 
-Tolerances (the benchmark spec's, restated in the design doc):
+Tolerances:
   * y: relative L2 <= 1e-5 per step;
   * state: <= 0.1% of codes differ, by 1 only outside a re-scaled column;
     row factors / column scales differ in <= 0.1% of rows / columns.
-This build meets the state contract with no difference at all (the tests
+The kernels meet the state contract with no difference at all (the tests
 assert identical bytes), because delta, X and the column objective are
 evaluated in the oracle's order.
 """
