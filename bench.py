@@ -65,22 +65,29 @@ MODES = {
     "spatial": (W.MODE_STEPQUANT, 6, False),
     "temporal": (W.MODE_UNIFORM, None, True),
     "nopivot": (W.MODE_STEPQUANT, None, False),
-    "calibrated": (W.MODE_STEPQUANT, None, True),   # widths from calibrated_plan()
+    # offline calibration (calibrated_plan): estimated row-impact weights,
+    # allocated widths, or both
+    "impact": (W.MODE_STEPQUANT, None, True),
+    "allocated": (W.MODE_STEPQUANT, None, True),
+    "calibrated": (W.MODE_STEPQUANT, None, True),
 }
 
 CAL_STEPS, CAL_SNAPSHOTS, CAL_REQUESTS = 64, 4, 16
 CAL_STEP_BASE = 1 << 24     # calibration inputs: step indices no decode run uses
 
 
-def calibrated_plan(cfg):
-    """The workload's plan with widths and pivots from the lifetime-aware
-    allocation, calibrated on fp32 rollouts of held-out requests and steps.
+def calibrated_plan(cfg, what):
+    """The workload's plan with calibrated row-impact weights ("impact"),
+    widths and pivots from the lifetime-aware allocation ("allocated"), or
+    both ("calibrated": the weights first, then the allocation measured with
+    them).
 
-    Calibration states: CAL_REQUESTS requests numbered after the workload's
-    own, stepped CAL_STEPS times by the fp32 kernel from their seeded S0 with
-    seeded inputs of step indices CAL_STEP_BASE + t, snapshotted CAL_SNAPSHOTS
-    times; lifetimes from the plan's gates; the budget and the pivot count of
-    the workload's own recipe."""
+    Calibration data: CAL_REQUESTS requests numbered after the workload's own,
+    stepped CAL_STEPS times by the fp32 kernel from their seeded S0 with
+    seeded inputs of step indices CAL_STEP_BASE + t; the row-impact scores
+    from every step's inputs, the distortion from CAL_SNAPSHOTS snapshots of
+    the states; lifetimes from the plan's gates; the budget and the pivot
+    count of the workload's own recipe."""
     import torch
 
     import quantized_delta_rule_decode_b200 as S
@@ -92,31 +99,36 @@ def calibrated_plan(cfg):
     slots = torch.arange(len(reqs), dtype=torch.int32, device="cuda")
     dt = torch.bfloat16 if cfg.bf16_inputs else torch.float32
     y = torch.empty((len(reqs), H, d), dtype=torch.float32, device="cuda")
-    states = []
+    states, inputs = [], []
     every = CAL_STEPS // CAL_SNAPSHOTS
     for t in range(CAL_STEPS):
         si = W.step_inputs(cfg, CAL_STEP_BASE + t, pin, reqs)
         q, k, v = (torch.from_numpy(a).to(dt).cuda() for a in (si.q, si.k, si.v))
         beta, gate = torch.from_numpy(si.beta).cuda(), torch.from_numpy(si.gate).cuda()
+        inputs.append((q, k, beta, gate))
         S.stepq_fp32_step(Sx, slots, q, k, v, beta, gate, y, cfg.gate_kind)
         if (t + 1) % every == 0:
             states.append(Sx.clone())
-    g = np.asarray(pin.gate, np.float32)
-    if cfg.unit_kind == W.UNIT_ROW:
-        g = g.reshape(-1) if cfg.gate_kind == W.GATE_DIAG else np.repeat(g, d)
-    elif g.ndim == 2:
-        g = None
-    gates = g[None, :, None] if g is not None else np.asarray(pin.gate, np.float32)[None]
-    n_piv = int(np.sum(pin.bits == 16))
-    bits, _, _ = calibrate.calibrate_bits(d, d, H, cfg.gate_kind, cfg.unit_kind, pin.w, states, gates,
-                                          cfg.budget, n_piv)
-    return W.PlanInputs(bits=bits, w=pin.w, half_life=pin.half_life, gate=pin.gate)
+    w = pin.w
+    if what in ("impact", "calibrated"):
+        w = calibrate.impact_weights(cfg.gate_kind, d, H, inputs)
+    bits = pin.bits
+    if what in ("allocated", "calibrated"):
+        g = np.asarray(pin.gate, np.float32)
+        if cfg.unit_kind == W.UNIT_ROW:
+            gates = (g.reshape(-1) if cfg.gate_kind == W.GATE_DIAG else np.repeat(g, d))[None, :, None]
+        else:
+            gates = g[None] if g.ndim == 2 else g[None, :, None]
+        n_piv = int(np.sum(pin.bits == 16))
+        bits, _, _ = calibrate.calibrate_bits(d, d, H, cfg.gate_kind, cfg.unit_kind, w, states, gates,
+                                              cfg.budget, n_piv)
+    return W.PlanInputs(bits=bits, w=w, half_life=pin.half_life, gate=pin.gate)
 
 
 def mode_plan(cfg, mode):
     m, ub, piv = MODES[mode]
-    if mode == "calibrated":
-        return m, calibrated_plan(cfg)
+    if mode in ("impact", "allocated", "calibrated"):
+        return m, calibrated_plan(cfg, mode)
     return m, W.make_plan(cfg, uniform_bits=ub, pivots=piv)
 
 
@@ -138,7 +150,7 @@ def parse():
                     help="skip the CUDA-graph replay of the same steps")
     ap.add_argument("--drift", action="store_true",
                     help="instead of the throughput line: quantised rollouts vs the fp32 rollout")
-    ap.add_argument("--drift-arms", default="stepquant,calibrated,uniform8,uniform6",
+    ap.add_argument("--drift-arms", default="stepquant,impact,allocated,calibrated,temporal,uniform8,uniform6",
                     help="comma-separated quantiser variants of the drift report")
     ap.add_argument("--drift-steps", type=int, default=0,
                     help="steps of the drift report (0: the workload's own step count)")

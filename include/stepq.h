@@ -336,6 +336,40 @@ STEPQ_API int stepq_lifetime_weight(int64_t n_units, int64_t n_steps, int32_t ga
 STEPQ_API int stepq_allocate_bits(int64_t n_units, const double *weight, const double *dist,
                                   int32_t budget_bits, int64_t n_pivots, uint8_t *bits);
 
+/* ------------------------------------------------------------------------
+ * Offline calibration: row-impact weights.  hyper.ai summary, section
+ * "Method", the paragraphs on the spatial distribution of errors and on
+ * key-row-aware dual-axis fitting: the impact of a key row is the expectation,
+ * over calibration tokens, of the square of the factor through which an error
+ * in that row reaches the readout; it weights the row factors and the column
+ * fit (the plan's w).
+ * ------------------------------------------------------------------------ */
+
+/* Add, for every (head, key row), the squared weighting factor over n
+ * calibration inputs (requests x tokens):
+ *     score_sum[h][i] += sum_r ((A_r^T q_r)_i)^2,
+ *     A_r = (I - beta_r k_r k_r^T) D_r   (the transition of the step that
+ *     reads the stored state), i.e. (A^T q)_i = g_i (q_i - beta k_i (k . q)).
+ *   q, k       device, [n][n_heads][d_k] in qkv_dtype (STEPQ_DTYPE_F32 / _BF16)
+ *   beta       device, fp32 [n][n_heads]
+ *   gate       device, fp32 [n][n_heads] (STEPQ_GATE_SCALAR) or
+ *              [n][n_heads][d_k] (STEPQ_GATE_DIAG)
+ *   score_sum  device, float64 [n_heads][d_k], read and written (caller zeroes
+ *              it before the first call)
+ * Arithmetic in double from the input values; per head the inputs are taken
+ * in ascending order.  Asynchronous on `stream`; d_k in {64, 128}. */
+STEPQ_API int stepq_row_impact(int32_t d_k, int32_t n_heads, int32_t gate_kind, int32_t qkv_dtype,
+                               int64_t n, const void *q, const void *k, const float *beta,
+                               const float *gate, double *score_sum, void *stream);
+
+/* The plan's row-impact weights from the accumulated scores:
+ * w[i] = sqrt(score_sum[i] / count), rounded to fp32, so that the column fit's
+ * weight w^2 is the mean squared weighting factor.
+ *   score_sum  host, float64 [n_rows]; every entry finite and > 0
+ *   w          host, fp32 [n_rows] (written)
+ * Host-only.  STEPQ_ERR_INVALID on bad arguments (nothing written). */
+STEPQ_API int stepq_impact_weights(int64_t n_rows, int64_t count, const double *score_sum, float *w);
+
 /* Synchronously read the pool's device status word (STEPQ_DEV_* bits, OR-ed
  * over every call since the last clear).  Waits for the device to go idle. */
 STEPQ_API int stepq_get_status(stepq_pool *pool, uint32_t *out);

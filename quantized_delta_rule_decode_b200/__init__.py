@@ -35,11 +35,13 @@ from ._ffi import (  # noqa: F401
     stepq_fp32_step,
     stepq_get_status,
     stepq_host_workspace_bytes,
+    stepq_impact_weights,
     stepq_lifetime_weight,
     stepq_pack,
     stepq_plan_create,
     stepq_plan_destroy,
     stepq_plan_head_layout,
+    stepq_row_impact,
     stepq_unit_distortion,
     stepq_plan_slot_bytes,
     stepq_pool_alloc,

@@ -40,6 +40,8 @@ _SIGS = {
     "stepq_unit_distortion": [_P, _P, _P, _I64, _P, _P, _P],
     "stepq_lifetime_weight": [_I64, _I64, _I32, _P, _P],
     "stepq_allocate_bits": [_I64, _P, _P, _I32, _I64, _P],
+    "stepq_row_impact": [_I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P],
+    "stepq_impact_weights": [_I64, _I64, _P, _P],
     "stepq_get_status": [_P, ctypes.POINTER(ctypes.c_uint32)],
     "stepq_clear_status": [_P, _P],
     "stepq_last_error": [],
@@ -327,6 +329,24 @@ def stepq_allocate_bits(weight, dist, budget_bits: int, n_pivots: int) -> np.nda
     _call("stepq_allocate_bits", w.size, w.ctypes.data_as(_P), d.ctypes.data_as(_P), int(budget_bits),
           int(n_pivots), bits.ctypes.data_as(_P))
     return bits
+
+
+def stepq_row_impact(gate_kind, q, k, beta, gate, score_sum, stream=None):
+    """score_sum [n_heads][d_k] float64 (device) += squared readout weighting factors of q, k."""
+    import torch
+    n, H, dk = q.shape
+    _call("stepq_row_impact", dk, H, gate_kind, _qkv_dtype(q), n, _ptr(q, q.dtype, "q"),
+          _ptr(k, q.dtype, "k"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
+          _ptr(score_sum, torch.float64, "score_sum"), _stream(stream))
+    return score_sum
+
+
+def stepq_impact_weights(score_sum, count: int) -> np.ndarray:
+    """Host float64 sums [n_rows] -> fp32 weights sqrt(sum / count)."""
+    s = np.ascontiguousarray(score_sum, np.float64).reshape(-1)
+    w = np.zeros(s.size, np.float32)
+    _call("stepq_impact_weights", s.size, int(count), s.ctypes.data_as(_P), w.ctypes.data_as(_P))
+    return w
 
 
 def stepq_get_status(pool: Pool) -> int:

@@ -1,9 +1,14 @@
-"""Offline lifetime-aware bit allocation, driven through the C ABI.
+"""Offline calibration of a plan, driven through the C ABI.
 
-hyper.ai summary of the paper, section "Method" (the Lifetime-Aware Bit
-Allocation paragraph); rcap.io post, "Temporal" part.  Before decoding, every
-state unit (a head, or one key row) gets its width:
+hyper.ai summary of the paper, section "Method" (the paragraphs on
+Lifetime-Aware Bit Allocation and on the spatial distribution of errors);
+rcap.io post, "Temporal" part and the sentence placing calibration offline.
+Before decoding, every key row gets its impact weight and every state unit
+(a head, or one key row) its width:
 
+0. the plan's row-impact weights from the calibration inputs
+   (``stepq_row_impact``, ``stepq_impact_weights``; hyper.ai, the paragraph on
+   the spatial distribution of errors);
 1. quantise calibration states with a plan of one width b for every unit
    (b = 4, 6, 8; the full quantiser: row factors, dual-axis fit) and measure
    each unit's squared reconstruction error (``stepq_unit_distortion``);
@@ -21,11 +26,32 @@ from __future__ import annotations
 
 import numpy as np
 
-from ._ffi import (MODE_STEPQUANT, UNIT_ROW, stepq_allocate_bits, stepq_lifetime_weight,
-                   stepq_pack, stepq_plan_create, stepq_pool_alloc, stepq_plan_slot_bytes,
-                   stepq_unit_distortion)
+from ._ffi import (MODE_STEPQUANT, UNIT_ROW, stepq_allocate_bits, stepq_impact_weights,
+                   stepq_lifetime_weight, stepq_pack, stepq_plan_create, stepq_pool_alloc,
+                   stepq_plan_slot_bytes, stepq_row_impact, stepq_unit_distortion)
 
 WIDTHS = (4, 6, 8)
+
+
+def impact_weights(gate_kind, d_k, n_heads, inputs, stream=None) -> np.ndarray:
+    """The plan's row-impact weights w [n_heads][d_k] from calibration inputs.
+
+    hyper.ai summary, section "Method" (the paragraph on the spatial
+    distribution of errors): a key row's impact score is the mean square of
+    the factor through which its error reaches the readout; the weight is its
+    square root.  inputs: iterable of device (q, k, beta, gate) in the decode
+    step's layouts ([n][n_heads][d_k], [n][n_heads], gate per head or row)."""
+    import torch
+    score = None
+    count = 0
+    for q, k, beta, gate in inputs:
+        if score is None:
+            score = torch.zeros((n_heads, d_k), dtype=torch.float64, device=q.device)
+        stepq_row_impact(gate_kind, q, k, beta, gate, score, stream=stream)
+        count += q.shape[0]
+    if score is None:
+        raise ValueError("no calibration inputs")
+    return stepq_impact_weights(score.cpu().numpy(), count).reshape(n_heads, d_k)
 
 
 def measure_distortion(d_k, d_v, n_heads, gate_kind, unit_kind, w, states, stream=None):

@@ -1,5 +1,7 @@
-// Offline lifetime-aware bit allocation: host code behind
-// stepq_lifetime_weight and stepq_allocate_bits.
+// Offline calibration, host code: stepq_lifetime_weight and
+// stepq_allocate_bits (lifetime-aware bit allocation, below) and
+// stepq_impact_weights (the plan's row-impact weights from the scores that
+// the row-impact kernel accumulates: w = sqrt(mean squared weighting factor)).
 //
 // hyper.ai summary of the paper, section "Method" (the Lifetime-Aware Bit
 // Allocation paragraph): per state unit, the reconstruction distortion at
@@ -52,6 +54,17 @@ extern "C" int stepq_lifetime_weight(int64_t n_units, int64_t n_steps, int32_t g
         const double ell = acc / count;  // mean log retention, < 0
         weight[u] = 1.0 / (1.0 - std::exp(ell));
     }
+    return STEPQ_OK;
+}
+
+extern "C" int stepq_impact_weights(int64_t n_rows, int64_t count, const double *score_sum, float *w) {
+    stepq::set_error(STEPQ_OK, "");
+    if (n_rows <= 0 || count <= 0) return invalid("n_rows and count must be positive");
+    if (!score_sum || !w) return invalid("score_sum and w must not be NULL");
+    for (int64_t i = 0; i < n_rows; ++i)
+        if (!(std::isfinite(score_sum[i]) && score_sum[i] > 0.0))
+            return invalid("every score sum must be finite and > 0 (a row that never reaches the readout)");
+    for (int64_t i = 0; i < n_rows; ++i) w[i] = float(std::sqrt(score_sum[i] / double(count)));
     return STEPQ_OK;
 }
 

@@ -527,6 +527,28 @@ int stepq_decode_step_host(const stepq_plan *plan, stepq_pool *pool, const int32
     return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "device-to-host copy");
 }
 
+int stepq_row_impact(int32_t d_k, int32_t n_heads, int32_t gate_kind, int32_t qkv_dtype, int64_t n,
+                     const void *q, const void *k, const float *beta, const float *gate,
+                     double *score_sum, void *stream) {
+    g_err.clear();
+    if (d_k != 64 && d_k != 128) return fail(STEPQ_ERR_UNSUPPORTED, "the library runs d_k in {64, 128}");
+    if (n_heads <= 0 || n_heads > 65535) return fail(STEPQ_ERR_INVALID, "n_heads must be in [1, 65535]");
+    if (gate_kind != STEPQ_GATE_SCALAR && gate_kind != STEPQ_GATE_DIAG)
+        return fail(STEPQ_ERR_INVALID, "gate_kind %d unknown", gate_kind);
+    if (qkv_dtype != STEPQ_DTYPE_F32 && qkv_dtype != STEPQ_DTYPE_BF16)
+        return fail(STEPQ_ERR_INVALID, "qkv_dtype %d unknown", qkv_dtype);
+    if (n < 0) return fail(STEPQ_ERR_INVALID, "n must be >= 0");
+    int rc;
+    if ((rc = check_inputs(score_sum, "score_sum"))) return rc;
+    if (n == 0) return STEPQ_OK;
+    if ((rc = check_inputs(q, "q")) || (rc = check_inputs(k, "k")) || (rc = check_inputs(beta, "beta")) ||
+        (rc = check_inputs(gate, "gate")))
+        return rc;
+    cudaError_t e = stepq::launch_row_impact(d_k, n_heads, gate_kind, qkv_dtype, n, q, k, beta, gate,
+                                             score_sum, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "row impact launch");
+}
+
 int stepq_fp32_step(int32_t d_k, int32_t d_v, int32_t n_heads, int32_t gate_kind,
                     int32_t qkv_dtype, float *S, int64_t num_slots, const int32_t *slot_idx,
                     int64_t n, const void *q, const void *k, const void *v, const float *beta,

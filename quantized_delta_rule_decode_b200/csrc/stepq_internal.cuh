@@ -61,6 +61,9 @@ cudaError_t launch_fitpack(const PlanDev &P, const StepArgs &a, int qkv_dtype, c
 cudaError_t launch_pack(const PlanDev &P, const StepArgs &a, cudaStream_t s);
 cudaError_t launch_unpack(const PlanDev &P, const StepArgs &a, cudaStream_t s);
 cudaError_t launch_distortion(const PlanDev &P, const StepArgs &a, cudaStream_t s);
+cudaError_t launch_row_impact(int d, int H, int gate_kind, int qkv, int64_t n, const void *q,
+                              const void *k, const float *beta, const float *gate, double *score,
+                              cudaStream_t s);
 cudaError_t launch_fp32_step(int d, int H, int gate_kind, int qkv_dtype, float *S, int64_t num_slots,
                              const int32_t *slot_idx, int64_t n, const void *q, const void *k,
                              const void *v, const float *beta, const float *gate, float *y,

@@ -94,3 +94,28 @@ def test_calibration_matches_oracle(name):
     rest = bits[bits != 16]
     assert np.sum(rest, dtype=np.int64) <= budget * rest.size
     assert np.sum(bits == 16) == n_piv
+
+
+@pytest.mark.parametrize("name", ["gdn", "kda", "tiny"])
+def test_row_impact_matches_oracle(name):
+    """Row-impact scores (hyper.ai, Method: the spatial paragraph): two
+    accumulating calls over 3 requests each, against the oracle's float64 sums."""
+    import torch
+
+    from oracle import impact as I
+    from gpu_harness import step_tensors
+    cfg = W.CONFIGS[name]
+    pin = W.make_plan(cfg)
+    S = lib()
+    reqs = [0, 1, 2]
+    score = torch.zeros((cfg.heads, cfg.d), dtype=torch.float64, device="cuda")
+    want = np.zeros((cfg.heads, cfg.d))
+    for step in (0, 1):
+        si = W.step_inputs(cfg, step, pin, reqs)
+        t = step_tensors(cfg, si)
+        S.stepq_row_impact(cfg.gate_kind, t["q"], t["k"], t["beta"], t["gate"], score)
+        want += I.score_sum(si.q, si.k, si.beta, si.gate, cfg.gate_kind)
+    torch.cuda.synchronize()
+    assert np.allclose(score.cpu().numpy(), want, rtol=1e-12, atol=0)
+    w = S.stepq_impact_weights(score.cpu().numpy(), 2 * len(reqs))
+    assert np.allclose(w, I.impact_weights(want, 2 * len(reqs)).reshape(-1), rtol=1e-6, atol=0)
