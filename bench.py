@@ -150,6 +150,8 @@ def parse():
                     help="skip the CUDA-graph replay of the same steps")
     ap.add_argument("--drift", action="store_true",
                     help="instead of the throughput line: quantised rollouts vs the fp32 rollout")
+    ap.add_argument("--pipeline", action="store_true",
+                    help="instead of the throughput line: per-token time of a layer stack with GEMM proxies")
     ap.add_argument("--drift-arms", default="stepquant,impact,allocated,calibrated,temporal,uniform8,uniform6",
                     help="comma-separated quantiser variants of the drift report")
     ap.add_argument("--drift-steps", type=int, default=0,
@@ -713,6 +715,87 @@ def run_drift(args, dist):
         print(json.dumps(out), flush=True)
 
 
+PIPE_HIDDEN = 5120          # model width of the projection proxy (a 27B-class hybrid model)
+
+
+def run_pipeline(args, dist):
+    """Per-token critical path of a stack of layers (rcap.io post, the sentence
+    after the pseudocode; hyper.ai summary, "Method", last paragraph: the fit
+    and pack run on a separate stream, overlapped with later-layer compute).
+
+    One token = L layers; each layer on the main stream: an input projection
+    GEMM [R, hidden] x [hidden, 3 H d] (bf16, cuBLAS through torch), the
+    readout kernel, an output projection GEMM [R, H d] x [H d, hidden]; the
+    layer's fit + pack on the side stream after its readout.  The GEMMs stand
+    in for the model's own compute (their outputs are not fed to the state
+    step, which reads the seeded ring of inputs).  Variants: the two-stream
+    design, the fit on the main stream, the GEMMs alone, and the fp32-state
+    step in place of the quantised one.  Device time with CUDA events over K
+    tokens after W warm-up tokens."""
+    import torch
+    cfg = W.CONFIGS[args.config]
+    wl = DeviceWorkload(cfg, args.mode)
+    L = wl.layers
+    R, H, d = cfg.requests, cfg.heads, cfg.d
+    hid = PIPE_HIDDEN
+    g = torch.Generator(device="cuda").manual_seed(7)
+    w_in = [torch.randn((hid, 3 * H * d), device="cuda", dtype=torch.bfloat16, generator=g) * 0.01
+            for _ in range(L)]
+    w_out = [torch.randn((H * d, hid), device="cuda", dtype=torch.bfloat16, generator=g) * 0.01
+             for _ in range(L)]
+    x = torch.randn((R, hid), device="cuda", dtype=torch.bfloat16, generator=g)
+    y_in = torch.empty((R, 3 * H * d), device="cuda", dtype=torch.bfloat16)
+    o_in = torch.randn((R, H * d), device="cuda", dtype=torch.bfloat16, generator=g)
+    x_out = torch.empty((R, hid), device="cuda", dtype=torch.bfloat16)
+    P = ctypes.c_void_p
+    ms = P(wl.main.cuda_stream)
+    # fp32 state per layer for the unquantised variant
+    S32 = [torch.zeros((cfg.pool_slots, H, d, d), dtype=torch.float32, device="cuda") for _ in range(L)]
+    t0 = wl.ring[0]
+    y32 = torch.empty((R, H, d), dtype=torch.float32, device="cuda")
+
+    def token(tok, variant):
+        for l in range(L):
+            torch.matmul(x, w_in[l], out=y_in)
+            i = l * 16 + tok % 16
+            if variant == "two_streams":
+                if wl.L.stepq_decode_step(*wl.step_args[i]):
+                    raise RuntimeError(wl.L.stepq_last_error().decode())
+            elif variant == "one_stream":
+                a = list(wl.step_args[i])
+                a[-1] = ms
+                if wl.L.stepq_decode_step(*a):
+                    raise RuntimeError(wl.L.stepq_last_error().decode())
+            elif variant == "fp32_state":
+                wl.S.stepq_fp32_step(S32[l], wl.slots, t0["q"], t0["k"], t0["v"], t0["beta"], t0["gate"],
+                                     y32, cfg.gate_kind)
+            torch.matmul(o_in, w_out[l], out=x_out)
+
+    out = {}
+    for variant in ("two_streams", "one_stream", "gemm_only", "fp32_state"):
+        for tok in range(args.warmup):
+            token(tok, variant)
+        wl.join()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(wl.main)
+        for tok in range(args.steps):
+            token(tok, variant)
+        wl.join()
+        b.record(wl.main)
+        torch.cuda.synchronize()
+        out[variant] = dist.max(a.elapsed_time(b) / args.steps)
+    gemm = out["gemm_only"]
+    line = {"report": "per-token critical path of a layer stack (GEMM proxy + state step)",
+            "config": args.config, "mode": args.mode, "layers": L, "requests": R, "hidden": hid,
+            "tokens": args.steps, "warmup": args.warmup, "data": "synthetic (seeded; workload.py)",
+            "ms_per_token": out,
+            "state_step_ms_per_layer": {k: (v - gemm) / L for k, v in out.items() if k != "gemm_only"},
+            "overlap_saved_ms_per_token": out["one_stream"] - out["two_streams"]}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def cpu_model():
     try:
         for line in open("/proc/cpuinfo"):
@@ -801,10 +884,10 @@ def main():
         run_reference(args, dist)
         dist.close()
         return
-    if args.drift:
+    if args.drift or args.pipeline:
         import torch
         torch.cuda.set_device(dist.local)
-        run_drift(args, dist)
+        (run_drift if args.drift else run_pipeline)(args, dist)
         dist.close()
         return
     import torch
