@@ -16,8 +16,11 @@ import subprocess
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "stepq_oracle.c")
-_LIB = os.path.join(_HERE, "liboracle_stepq.so")
+# STEPQ_ORACLE_SRC / STEPQ_ORACLE_LIB: build and load another copy of the
+# source instead (the mutation test plants mistakes in copies to check that
+# the pins catch them)
+_SRC = os.environ.get("STEPQ_ORACLE_SRC", os.path.join(_HERE, "stepq_oracle.c"))
+_LIB = os.environ.get("STEPQ_ORACLE_LIB", os.path.join(_HERE, "liboracle_stepq.so"))
 _CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
 
 
