@@ -806,9 +806,7 @@ def cpu_model():
     return "unknown"
 
 
-def run_reference(args, dist):
-    if dist.rank != 0:
-        return
+def run_reference(args):
     cfg = W.CONFIGS[args.config]
     orc = OracleRunner(cfg, args.mode)
     warm_rate, _ = orc.rate(2.0)
@@ -879,11 +877,12 @@ def ncu_traffic(kernel, workload):
 
 def main():
     args = parse()
-    dist = Dist(args.gpus)
     if args.impl == "reference":
-        run_reference(args, dist)
-        dist.close()
+        # the oracle on the host: rank 0 alone, no process group and no GPU
+        if int(os.environ.get("RANK", "0")) == 0:
+            run_reference(args)
         return
+    dist = Dist(args.gpus)
     if args.drift or args.pipeline:
         import torch
         torch.cuda.set_device(dist.local)

@@ -77,3 +77,22 @@ def test_two_ranks_shard_requests_without_exchange():
         for a, r in enumerate(part["reqs"]):
             assert np.array_equal(part["y"][a], y[r])
             assert np.array_equal(part["pool"][a * sb:(a + 1) * sb], pool[r * sb:(r + 1) * sb])
+
+
+@pytest.mark.timeout(600)
+def test_reference_arm_under_torchrun_prints_once():
+    """bench.py --impl reference launched as the two-rank job: rank 0 alone
+    times the oracle and prints one line; every rank exits 0."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                        "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py",
+                        "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                       cwd=root, capture_output=True, text=True, timeout=500)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
