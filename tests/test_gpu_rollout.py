@@ -8,7 +8,8 @@ runs in full on the GPU, in the launch configuration bench.py times, and is
 compared on a fixed subset of 2 requests x 16 heads.  Since the kernels
 evaluate delta, X and the column objective in the oracle's order, the
 rollouts stay identical, and the tests also check the packed bytes (every step for the
-short rollouts).
+short rollouts) and the readout y of every step (relative L2 <= 1e-5, the
+one-step bound).
 """
 
 from concurrent.futures import ThreadPoolExecutor
@@ -61,6 +62,10 @@ def _rollout(name, steps, compare_reqs, gpu_reqs, mode=W.MODE_STEPQUANT, ub=None
             yo[key] = yy
 
         list(ex.map(one, keys))
+        # the readout of every step, against the oracle's
+        yg = y.cpu().numpy()
+        worst_y = max(worst_y, rel_l2(np.array([yg[r, h] for (r, h) in keys]),
+                                      np.array([yo[key] for key in keys])))
         if bytes_every and (step % bytes_every == bytes_every - 1 or step == steps - 1):
             # the packed slots, byte for byte: a transient divergence (one row
             # factor off by a half ulp for one step) cannot pass unseen
@@ -76,8 +81,7 @@ def _rollout(name, steps, compare_reqs, gpu_reqs, mode=W.MODE_STEPQUANT, ub=None
             for r in compare_reqs:
                 d = rel_l2(gS[r], oS[r])
                 worst_drift = max(worst_drift, d)
-            yg = y.cpu().numpy()
-            worst_y = max(worst_y, max(rel_l2(yg[r, h], yo[(r, h)]) for (r, h) in keys))
+
     ex.shutdown()
     assert S.stepq_get_status(pool) == 0
     return worst_drift, worst_y
@@ -86,21 +90,25 @@ def _rollout(name, steps, compare_reqs, gpu_reqs, mode=W.MODE_STEPQUANT, ub=None
 def test_rollout_tiny_256_steps():
     drift, ydiff = _rollout("tiny", 256, [0], 1, every=8, bytes_every=1)
     assert drift <= 1e-3, drift
+    assert ydiff <= 1e-5, ydiff
 
 
 def test_rollout_tiny_uniform8_256_steps():
-    drift, _ = _rollout("tiny", 256, [0], 1, mode=W.MODE_UNIFORM, ub=8, every=16, bytes_every=1)
+    drift, ydiff = _rollout("tiny", 256, [0], 1, mode=W.MODE_UNIFORM, ub=8, every=16, bytes_every=1)
     assert drift <= 1e-3, drift
+    assert ydiff <= 1e-5, ydiff
 
 
 def test_rollout_kda_256_steps():
     """Per-key-row gates and widths (with FP16 pivot rows), 2 requests."""
-    drift, _ = _rollout("kda", 256, [0, 1], 2, every=64, bytes_every=1)
+    drift, ydiff = _rollout("kda", 256, [0, 1], 2, every=64, bytes_every=1)
     assert drift <= 1e-3, drift
+    assert ydiff <= 1e-5, ydiff
 
 
 @pytest.mark.slow
 def test_rollout_long_4096_steps_subset():
     """128 requests x 16 heads on the GPU for 4096 steps; 2 x 16 compared."""
-    drift, _ = _rollout("rollout", 4096, [0, 1], 128, every=256, bytes_every=256)
+    drift, ydiff = _rollout("rollout", 4096, [0, 1], 128, every=256, bytes_every=256)
     assert drift <= 1e-3, drift
+    assert ydiff <= 1e-5, ydiff
