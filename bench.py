@@ -31,6 +31,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -856,10 +857,14 @@ def workload_config(cfg, mode, wl):
 
 
 def src_sha():
-    """Hash of the sources that define the device kernels (not the host API)."""
+    """Hash of the code (comments and spacing removed) that defines the device
+    kernels, not the host API."""
     h = hashlib.sha256()
     for f in ("stepq_kernels.cu", "stepq_internal.cuh"):
-        h.update(open(os.path.join(ROOT, "quantized_delta_rule_decode_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "quantized_delta_rule_decode_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 
