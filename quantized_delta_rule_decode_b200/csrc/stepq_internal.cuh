@@ -72,6 +72,6 @@ cudaError_t launch_fp32_step(int d, int H, int gate_kind, int qkv_dtype, float *
 
 // Record an error message for stepq_last_error(); returns code.
 int set_error(int code, const char *msg);
-size_t quant_smem_bytes(int d, uint32_t max_qhead_bytes);
+size_t quant_smem_bytes(int d);
 
 }  // namespace stepq
