@@ -46,9 +46,13 @@ class Pair:
     """A plan on both sides, from one workload config."""
 
     def __init__(self, cfg: W.Config, mode=W.MODE_STEPQUANT, uniform_bits=None, budget=None,
-                 pivots=True):
+                 pivots=True, bits=None):
         self.cfg = cfg
         self.pin = W.make_plan(cfg, budget=budget, uniform_bits=uniform_bits, pivots=pivots)
+        if bits is not None:
+            # a hand-made width per unit instead of the synthetic plan's
+            import dataclasses
+            self.pin = dataclasses.replace(self.pin, bits=np.asarray(bits, np.uint8).reshape(-1))
         self.mode = mode
         d, H = cfg.d, cfg.heads
         S = lib()
