@@ -66,6 +66,17 @@ def test_pivots_are_the_largest_risks_ties_to_lower_index():
     assert list(np.nonzero(bits == 16)[0]) == [0, 1]
 
 
+def test_pivot_risk_is_taken_at_the_budget_width():
+    # the risk of a unit is its lifetime weight times its distortion at the
+    # budget width; the three widths rank these units differently:
+    #   at 4 bits 10, 10, 12 -> unit 2;  at 6 bits 5, 4, 3 -> unit 0;  at 8 bits 1, 3, 2 -> unit 1
+    L = np.ones(3)
+    D = np.array([[10.0, 5, 1], [10.0, 4, 3], [12.0, 3, 2]])
+    assert list(np.nonzero(A.allocate_bits(L, D, 6, 1) == 16)[0]) == [0]
+    assert list(np.nonzero(A.allocate_bits(L, D, 8, 1) == 16)[0]) == [1]
+    assert list(np.nonzero(A.allocate_bits(L, D, 4, 1) == 16)[0]) == [2]
+
+
 def test_equal_sums_give_the_earlier_unit_the_smaller_width():
     # two identical units, costs 3, 2, 1 (exact in binary): (4, 8), (6, 6) and
     # (8, 4) all sum to 4; the stated rule picks (4, 8)

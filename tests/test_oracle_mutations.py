@@ -2,10 +2,11 @@
 
 Each mutation below plants one mistake in a copy of oracle/stepq_oracle.c (a
 flipped sign, a dropped term, a transposed index, a wrong rounding, a wrong
-tie rule, a wrong bit order, ...).  The copy is built and the oracle's own pin
-tests are run against it in a subprocess; every mutant must make at least one
-of them fail.  A surviving mutant would mean a part of the oracle that nothing
-other than itself checks.
+tie rule, a wrong bit order, ...) or of the Python parts of the oracle (the
+bit allocation and the row-impact scores).  The copy is built and the
+oracle's own pin tests are run against it in a subprocess; every mutant must
+make at least one of them fail.  A surviving mutant would mean a part of the
+oracle that nothing other than itself checks.
 """
 
 import os
@@ -46,6 +47,30 @@ MUTATIONS = {
                         "double e = (double)Xh[i * dv + j] + (double)S[i * dv + j];"),
     "offset binary off by one": ("(uint32_t)(codes[i * dv + j] + (1 << (b - 1)))",
                                  "(uint32_t)(codes[i * dv + j] + (1 << (b - 1)) - 1)"),
+    "qmax off by one": ("qmax[i] = (1 << (b - 1)) - 1;", "qmax[i] = (1 << (b - 1));"),
+    "column max without the width factor": ("z = fabsf(X[i * dv + j]) * ikap[i];",
+                                            "z = fabsf(X[i * dv + j]) * irho[i];"),
+    "objective without the clamp": ("        if (q > two23 + (float)qmax[i])\n            q = two23 + (float)qmax[i];",
+                                    "        if (0)\n            q = two23 + (float)qmax[i];"),
+    "row factor over w, not sqrt(w)": ("float r = sqrtf(m) / sqrtf(pl->w[h * dk + i]);",
+                                       "float r = sqrtf(m) / pl->w[h * dk + i];"),
+    "objective weight not squared": (
+        "Aw[i] = (pl->w[h * dk + i] * orc_half_to_float(rho[i])) *\n"
+        "                        (pl->w[h * dk + i] * orc_half_to_float(rho[i]));",
+        "Aw[i] = pl->w[h * dk + i] * orc_half_to_float(rho[i]);"),
+    "objective scaled by c, not c^2": ("return (c * c) * ((P[0] + P[1]) + (P[2] + P[3]));",
+                                       "return c * ((P[0] + P[1]) + (P[2] + P[3]));"),
+    "uniform scale over qmax + 1": ("rho[i] = scale_half(m / (float)qmax[i]);",
+                                    "rho[i] = scale_half(m / (float)(qmax[i] + 1));"),
+    "codes clamped asymmetrically": ("if (r < -(float)qmax) r = -(float)qmax;",
+                                     "if (r < -(float)qmax - 1.0f) r = -(float)qmax - 1.0f;"),
+    "delta without beta": ("delta = beta * (v[j] - u);", "delta = (v[j] - u);"),
+    "update without k": ("X[i * dv + j] = g * S[i * dv + j] + k[i] * delta;",
+                         "X[i * dv + j] = g * S[i * dv + j] + delta;"),
+    "projection without the gate": ("u = u + k[i] * (g * S[i * dv + j]);   /* (k^T D S)_j */",
+                                    "u = u + k[i] * S[i * dv + j];   /* (k^T D S)_j */"),
+    "half rounding ties away": ("r = rintf(a / step) * step;", "r = roundf(a / step) * step;"),
+    "subnormal halves truncated": ("r = rintf(a * 0x1p24f) * 0x1p-24f;", "r = truncf(a * 0x1p24f) * 0x1p-24f;"),
 }
 
 
@@ -72,6 +97,68 @@ def test_every_planted_mistake_fails_a_pin():
     with tempfile.TemporaryDirectory() as tmp:
         with ThreadPoolExecutor(min(8, os.cpu_count() or 1)) as ex:
             results = list(ex.map(lambda kv: _run(kv[0], *kv[1], tmp), [CONTROL, *MUTATIONS.items()]))
+    assert results[0] == ("control", 0), f"the unmutated copy fails its pins: {results[0]}"
+    results = results[1:]
+    survivors = [name for name, rc in results if rc == 0]
+    errors = [(name, rc) for name, rc in results if rc not in (0, 1)]
+    assert not errors, f"pin runs that did not complete: {errors}"
+    assert not survivors, f"mutations no pin caught: {survivors}"
+
+
+# mistakes in the Python parts of the oracle: (module, old, new)
+PY_PINS = ["tests/test_oracle_alloc.py", "tests/test_oracle_impact.py"]
+PY_MUTATIONS = {
+    "lifetime weight without the geometric sum": (
+        "allocation.py", "out[u] = 1.0 / (1.0 - np.exp(ell))", "out[u] = np.exp(ell)"),
+    "log retention averaged over steps only": (
+        "allocation.py", "ell = acc / (steps * rows)", "ell = acc / steps"),
+    "pivots by lowest risk": (
+        "allocation.py", "key=lambda u: (-risk[u], u)", "key=lambda u: (risk[u], u)"),
+    "pivot risk at the widest width": ("allocation.py", "col = WIDTHS.index(budget)", "col = 2"),
+    "bit budget off by one": ("allocation.py", "K = N * (budget - 4) // 2", "K = N * (budget - 4) // 2 + 1"),
+    "ties to the wider width": ("allocation.py", "better = cand < best", "better = cand <= best"),
+    "backtracking loses the budget": ("allocation.py", "        k -= o", "        k -= min(o, 1)"),
+    "impact without the gate": ("impact.py", "om = g * (q[r, h, i] - beta[r, h] * k[r, h, i] * kq)",
+                                "om = (q[r, h, i] - beta[r, h] * k[r, h, i] * kq)"),
+    "impact with the wrong sign": ("impact.py", "om = g * (q[r, h, i] - beta[r, h] * k[r, h, i] * kq)",
+                                   "om = g * (q[r, h, i] + beta[r, h] * k[r, h, i] * kq)"),
+    "impact without beta": ("impact.py", "om = g * (q[r, h, i] - beta[r, h] * k[r, h, i] * kq)",
+                            "om = g * (q[r, h, i] - k[r, h, i] * kq)"),
+    "weights without the square root": ("impact.py", "np.sqrt(s / count).astype(np.float32)",
+                                        "(s / count).astype(np.float32)"),
+}
+
+
+def _run_py(name, module, old, new, tmp):
+    """The pins run from a directory whose oracle package holds the mutated
+    module; everything else is linked to the real files."""
+    d = os.path.join(tmp, name.replace(" ", "_"))
+    os.makedirs(os.path.join(d, "oracle"))
+    for f in os.listdir(os.path.join(ROOT, "oracle")):
+        if f == "__pycache__":
+            continue
+        os.symlink(os.path.join(ROOT, "oracle", f), os.path.join(d, "oracle", f))
+    src = open(os.path.join(ROOT, "oracle", module)).read()
+    assert src.count(old) == 1, f"mutation '{name}' does not apply"
+    os.remove(os.path.join(d, "oracle", module))
+    open(os.path.join(d, "oracle", module), "w").write(src.replace(old, new))
+    for f in ("tests", "workload.py", "quantized_delta_rule_decode_b200"):
+        os.symlink(os.path.join(ROOT, f), os.path.join(d, f))
+    env = dict(os.environ, PYTHONDONTWRITEBYTECODE="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", *PY_PINS, "-x", "-q", "-p", "no:cacheprovider",
+                        "-m", "not gpu"], cwd=d, env=env, capture_output=True, text=True, timeout=600)
+    return name, r.returncode
+
+
+def test_every_planted_mistake_in_the_python_oracle_fails_a_pin():
+    import oracle
+    oracle.build()
+    # control: an edit of a comment only
+    control = ("control", ("allocation.py", "# backward recurrence over the remaining units",
+                           "# the recurrence, from the last unit back"))
+    with tempfile.TemporaryDirectory() as tmp:
+        with ThreadPoolExecutor(min(8, os.cpu_count() or 1)) as ex:
+            results = list(ex.map(lambda kv: _run_py(kv[0], *kv[1], tmp), [control, *PY_MUTATIONS.items()]))
     assert results[0] == ("control", 0), f"the unmutated copy fails its pins: {results[0]}"
     results = results[1:]
     survivors = [name for name, rc in results if rc == 0]
