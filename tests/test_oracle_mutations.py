@@ -71,6 +71,26 @@ MUTATIONS = {
                                     "u = u + k[i] * S[i * dv + j];   /* (k^T D S)_j */"),
     "half rounding ties away": ("r = rintf(a / step) * step;", "r = roundf(a / step) * step;"),
     "subnormal halves truncated": ("r = rintf(a * 0x1p24f) * 0x1p-24f;", "r = truncf(a * 0x1p24f) * 0x1p-24f;"),
+    "reconstruction without the row scale": (
+        "S[i * dv + j] = (float)codes[i * dv + j] *\n"
+        "                                (orc_half_to_float(rho[i]) * orc_half_to_float(c[j]));",
+        "S[i * dv + j] = (float)codes[i * dv + j] *\n"
+        "                                (orc_half_to_float(c[j]));"),
+    "row maximum of signed values": ("float ax = fabsf(X[i * dv + j]);", "float ax = X[i * dv + j];"),
+    "non-finite rows not flagged": ("            if (bad) {\n                status |= ORC_STATUS_NONFINITE;",
+                                    "            if (bad) {\n                status |= 0;"),
+    "non-finite rows kept": ("            if (bad) {\n                status |= ORC_STATUS_NONFINITE;\n                m = 0.0f;",
+                             "            if (bad) {\n                status |= ORC_STATUS_NONFINITE;\n                m = m;"),
+    "pivot rows not flagged when non-finite": (
+        "                if (!isfinite(x))\n                    status |= ORC_STATUS_NONFINITE;\n"
+        "                piv[i * dv + j] = orc_float_to_half(x);",
+        "                if (!isfinite(x))\n                    status |= 0;\n"
+        "                piv[i * dv + j] = orc_float_to_half(x);"),
+    "readout with k for q": ("acc = acc + q[i] * X[i * dv + j];", "acc = acc + k[i] * X[i * dv + j];"),
+    "beta on the projection only": ("delta = beta * (v[j] - u);", "delta = v[j] - beta * u;"),
+    "distortion not squared": ("row += e * e;", "row += fabs(e);"),
+    "zero-column scale kept": ("                if (M == 0.0f) {\n                    c[j] = 0;",
+                               "                if (M == 0.0f) {\n                    c[j] = 0x3c00;"),
 }
 
 

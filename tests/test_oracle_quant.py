@@ -311,6 +311,30 @@ def test_zero_row_column_and_nonfinite(orc):
     assert rho2[7] == 0 and rho2[9] == 0 and np.all(codes2[7] == 0) and np.all(codes2[9] == 0)
 
 
+def test_nonfinite_pivot_rows_are_flagged(orc):
+    """A non-finite value in an FP16 pivot row is reported like one in a coded
+    row (the status word of the step), and is stored as the saturating half
+    conversion gives it (NaN -> 0, +-inf -> +-65504); the other rows are coded
+    as without it."""
+    rng = np.random.default_rng(51)
+    d = 16
+    X = _rand_X(rng, d, d)
+    bits = [6] * d
+    bits[4] = bits[11] = 16
+    plan = _make(orc, d, d, bits, np.ones(d, np.float32))
+    blob, st = plan.quantize_head(0, X)
+    assert st == 0
+    X2 = X.copy()
+    X2[4, 3] = np.nan
+    X2[11, 0] = -np.inf
+    blob2, st2 = plan.quantize_head(0, X2)
+    assert st2 & orc.STATUS_NONFINITE
+    codes, piv, rho, c = plan.unpack_codes(0, blob)
+    codes2, piv2, rho2, c2 = plan.unpack_codes(0, blob2)
+    assert piv2[4, 3] == 0 and piv2[11, 0] == np.float16(-65504.0).view(np.uint16)
+    assert np.array_equal(codes2, codes) and np.array_equal(rho2, rho) and np.array_equal(c2, c)
+
+
 @pytest.mark.parametrize("b", [4, 6, 8])
 def test_uniform_mode_absmax(orc, b):
     """The pages' uniform INT-b comparator: s_i = max_j|X_ij|/qmax, codes rne(X/s)."""
