@@ -91,6 +91,18 @@ MUTATIONS = {
     "distortion not squared": ("row += e * e;", "row += fabs(e);"),
     "zero-column scale kept": ("                if (M == 0.0f) {\n                    c[j] = 0;",
                                "                if (M == 0.0f) {\n                    c[j] = 0x3c00;"),
+    "halves big-endian": ("static void put_half(uint8_t *p, uint16_t h) { p[0] = (uint8_t)(h & 0xff); p[1] = (uint8_t)(h >> 8); }",
+                          "static void put_half(uint8_t *p, uint16_t h) { p[1] = (uint8_t)(h & 0xff); p[0] = (uint8_t)(h >> 8); }"),
+    "column scales before row scales": ("put_half(blob + pl->scale_off[h] + 2 * dk + 2 * j, c[j]);",
+                                        "put_half(blob + pl->scale_off[h] + 2 * j, c[j]);"),
+    "codes of a row packed from the wrong offset": ("put_bits(row, j * b, b, (uint32_t)(codes[i * dv + j] + (1 << (b - 1))));",
+                                                    "put_bits(row, j * b + 1, b, (uint32_t)(codes[i * dv + j] + (1 << (b - 1))));"),
+    "a positive scale may round to zero": ("    if (x > 0.0f && h == 0)\n        h = 1;",
+                                           "    if (x > 0.0f && h == 0)\n        h = 0;"),
+    "seven candidates": ("                for (a = 0; a < 8; a++) {\n                    uint16_t ca",
+                         "                for (a = 0; a < 7; a++) {\n                    uint16_t ca"),
+    "candidates over qmax of the row": ("uint16_t ca = scale_half((ALPHA[a] * M) / (float)qhi);",
+                                        "uint16_t ca = scale_half((ALPHA[a] * M) / (float)qmax[0]);"),
 }
 
 
