@@ -171,7 +171,7 @@ class Dist:
     The step has no exchange: ranks meet only at the timing barriers and for
     the max-over-ranks reduction of the measured times."""
 
-    def __init__(self, n=None, backend="nccl"):
+    def __init__(self, n=None, backend="nccl", timeout_s=120.0):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -184,7 +184,8 @@ class Dist:
             import torch.distributed as dist
             if backend == "nccl":
                 torch.cuda.set_device(self.local)
-            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            # a rank that is gone makes the others' next collective fail within this
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
             self.pg = dist
 
     def _device(self):

@@ -96,3 +96,44 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def _rank_that_leaves(rank, world, port, q):
+    """Rank 1 joins and leaves between steps (no collective in flight); rank 0
+    then reaches the timing barrier and must get an error, not hang."""
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "RANK": str(rank),
+                       "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank)})
+    import sys
+    import time
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    d = bench.Dist(backend="gloo", timeout_s=20.0)
+    d.barrier()                                      # both ranks are up
+    if rank == 1:
+        os._exit(0)                                  # gone without a word
+    time.sleep(1.0)
+    t0 = time.time()
+    try:
+        d.barrier()
+        d.max(1.0)
+        q.put(("no error", time.time() - t0))
+    except Exception as e:                           # noqa: BLE001 -- any backend error will do
+        q.put((type(e).__name__, time.time() - t0))
+    q.close()
+    q.join_thread()                                  # flushed before the hard exit below
+    os._exit(0)
+
+
+@pytest.mark.timeout(300)
+def test_a_rank_that_leaves_ends_the_next_collective_with_an_error():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_that_leaves, args=(r, world, port, q)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    outcome, waited = q.get(timeout=120)
+    for pr in procs:
+        pr.join(timeout=60)
+    assert outcome != "no error"
+    assert waited < 60.0                             # bounded by the process-group timeout
