@@ -18,7 +18,7 @@ from concurrent.futures import ThreadPoolExecutor
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "stepq_oracle.c")
 PINS = ["tests/test_oracle_half.py", "tests/test_oracle_pack.py", "tests/test_oracle_step.py",
-        "tests/test_oracle_quant.py", "tests/test_oracle_alloc.py"]
+        "tests/test_oracle_quant.py", "tests/test_oracle_alloc.py", "tests/test_oracle_fullsize_fit.py"]
 
 MUTATIONS = {
     "delta sign": ("delta = beta * (v[j] - u);", "delta = beta * (u - v[j]);"),
@@ -138,7 +138,7 @@ def test_every_planted_mistake_fails_a_pin():
 
 
 # mistakes in the Python parts of the oracle: (module, old, new)
-PY_PINS = ["tests/test_oracle_alloc.py", "tests/test_oracle_impact.py"]
+PY_PINS = ["tests/test_oracle_alloc.py", "tests/test_oracle_impact.py", "tests/test_oracle_fullsize_fit.py"]
 PY_MUTATIONS = {
     "lifetime weight without the geometric sum": (
         "allocation.py", "out[u] = 1.0 / (1.0 - np.exp(ell))", "out[u] = np.exp(ell)"),
@@ -158,6 +158,25 @@ PY_MUTATIONS = {
                             "om = g * (q[r, h, i] - k[r, h, i] * kq)"),
     "weights without the square root": ("impact.py", "np.sqrt(s / count).astype(np.float32)",
                                         "(s / count).astype(np.float32)"),
+    "definition: objective weight not squared": (
+        "definition.py", "w2 = np.asarray(w, np.float64) ** 2", "w2 = np.asarray(w, np.float64)"),
+    "definition: ties to the smaller alpha": (
+        "definition.py", "best = np.where(E[:, a] < E[np.arange(E.shape[0]), best], a, best)",
+        "best = np.where(E[:, a] <= E[np.arange(E.shape[0]), best], a, best)"),
+    "definition: candidate grid": ("definition.py", "(100 - 5 * a) / 100.0", "(100 - 4 * a) / 100.0"),
+    "definition: row factor times sqrt(w)": (
+        "definition.py", "r = np.sqrt(m) / np.sqrt(np.asarray(w, np.float64))",
+        "r = np.sqrt(m) * np.sqrt(np.asarray(w, np.float64))"),
+    "definition: codes truncated": ("definition.py", "q = np.clip(np.rint(t),", "q = np.clip(np.trunc(t),"),
+    "definition: column max without the width factor": (
+        "definition.py", "z = np.abs(X[active]) / rho[active, None] * (qhi / qmax[active])[:, None]",
+        "z = np.abs(X[active]) / rho[active, None]"),
+    "definition: half rounding through float32": (
+        "definition.py", "return x.astype(np.float16).view(np.uint16)",
+        "return x.astype(np.float32).astype(np.float16).view(np.uint16)"),
+    "definition: reconstruction without the row scale": (
+        "definition.py", "e = np.where(active[:, None], X - (rho[:, None] * ca[None, :]) * code, 0.0)",
+        "e = np.where(active[:, None], X - ca[None, :] * code, 0.0)"),
 }
 
 
