@@ -145,12 +145,19 @@ def parse():
     ap.add_argument("--fp32-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--kernel-steps", type=int, default=500,
+                    help="steps of the separate pass that times each kernel inside the overlapped step")
+    ap.add_argument("--config-steps", type=int, default=300,
+                    help="steps of each further workload measured into the line's 'configs' (0: none)")
     ap.add_argument("--isolated-steps", type=int, default=500,
                     help="steps of the per-kernel timing with each kernel alone")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="skip the CUDA-graph replay of the same steps")
     ap.add_argument("--drift", action="store_true",
                     help="instead of the throughput line: quantised rollouts vs the fp32 rollout")
+    ap.add_argument("--lifetime-study", action="store_true",
+                    help="instead of the throughput line: per-unit accumulated error of quantised rollouts "
+                         "vs the fp32 rollout, and its Spearman correlation with the unit's gate half-life")
     ap.add_argument("--pipeline", action="store_true",
                     help="instead of the throughput line: per-token time of a layer stack with GEMM proxies")
     ap.add_argument("--drift-arms", default="stepquant,impact,allocated,calibrated,temporal,uniform8,uniform6",
@@ -383,13 +390,14 @@ class DeviceWorkload:
 
 
 def time_device(wl, steps, warmup, dist, clocks_gpu):
+    """The headline: exactly `steps` plain stepq_decode_step calls between two
+    events on the main stream (joined with the side stream), barrier and
+    synchronize on both sides, max over ranks."""
     import torch
     for s in range(warmup):
         wl.run_step(s)
     wl.join()
     torch.cuda.synchronize()
-    stride = max(1, steps // 2000)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(0, steps, stride)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize()
@@ -397,20 +405,34 @@ def time_device(wl, steps, warmup, dist, clocks_gpu):
     time.sleep(0.3)
     start.record(wl.main)
     for s in range(steps):
-        if s % stride == 0:
-            wl.run_step_timed(warmup + s, evs[s // stride])
-        else:
-            wl.run_step(warmup + s)
+        wl.run_step(warmup + s)
     wl.join()
     end.record(wl.main)
     torch.cuda.synchronize()
     clocks = clk.stop()
     dist.barrier()
-    ms = start.elapsed_time(end)
-    ms = dist.max(ms)
+    ms = dist.max(start.elapsed_time(end))
+    return ms, clocks
+
+
+def time_kernels_overlapped(wl, steps, warmup):
+    """A separate pass after the headline: the same overlapped schedule with
+    CUDA events around each kernel on its own stream (the split calls
+    stepq_decode_readout + stepq_decode_fitpack), for the per-kernel durations
+    inside the step."""
+    import torch
+    for s in range(warmup):
+        wl.run_step(s)
+    wl.join()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for s in range(steps):
+        wl.run_step_timed(warmup + s, evs[s])
+    wl.join()
+    torch.cuda.synchronize()
     readout_ms = [e[0].elapsed_time(e[1]) for e in evs]
     fit_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    return ms, statistics.mean(readout_ms), statistics.mean(fit_ms), clocks
+    return statistics.mean(readout_ms), statistics.mean(fit_ms)
 
 
 def time_isolated(wl, steps, warmup):
@@ -717,6 +739,128 @@ def run_drift(args, dist):
         print(json.dumps(out), flush=True)
 
 
+def rank_average(x):
+    """1-based ranks of x, tied values sharing the mean of their ranks."""
+    x = np.asarray(x, np.float64)
+    order = np.argsort(x, kind="mergesort")
+    sx = x[order]
+    ranks = np.empty(x.size, np.float64)
+    i = 0
+    while i < x.size:
+        j = i
+        while j + 1 < x.size and sx[j + 1] == sx[i]:
+            j += 1
+        ranks[order[i:j + 1]] = (i + j) / 2.0 + 1.0
+        i = j + 1
+    return ranks
+
+
+def spearman_rho(a, b):
+    """Spearman rank correlation: the Pearson correlation of the two rank
+    vectors (average ranks for ties)."""
+    ra, rb = rank_average(a), rank_average(b)
+    ra -= ra.mean()
+    rb -= rb.mean()
+    den = math.sqrt(float(np.sum(ra * ra)) * float(np.sum(rb * rb)))
+    return float(np.sum(ra * rb) / den) if den > 0 else float("nan")
+
+
+LIFETIME_STUDIES = {
+    # units = heads: scalar per-head gates, half-lives log-uniform in [1, 4096]
+    "heads": dict(base="rollout", requests=8, heads=256),
+    # units = key rows: per-row gates and half-lives (KDA)
+    "rows": dict(base="kda", requests=16, heads=32),
+}
+
+
+def run_lifetime_study(args, dist):
+    """How a unit's accumulated quantisation error relates to its memory lifetime.
+
+    The pages find that a unit's gate half-life predicts how much INT6 error
+    it accumulates (Spearman rho about 0.80 over a model's heads; rcap.io
+    post, the "Temporal" paragraph; hyper.ai summary, Method, the lifetime
+    paragraph).  This is the synthetic analogue: quantised rollouts beside the
+    fp32 rollout of the same seeded inputs, for heads (scalar gates, one
+    half-life per head) and for key rows (KDA: one half-life per row).  Per
+    unit, the relative Frobenius error of its state against the fp32 state,
+    averaged over requests, at checkpoints; the reported "accumulated" error
+    is its mean over the checkpoints, and rho its Spearman rank correlation
+    with the unit's half-life, for uniform INT6, the workload's STEPQuant plan
+    (widths and pivots ranked by half-life) and the calibrated plan.
+    Reported, not checked: the pages measure this on real models."""
+    import dataclasses
+
+    import torch
+
+    import quantized_delta_rule_decode_b200 as S
+    steps = args.drift_steps or 2048
+    marks = [m for m in range(steps // 8, steps + 1, steps // 8)]
+    out = {"report": "lifetime vs accumulated quantisation error (synthetic analogue)", "steps": steps,
+           "checkpoints": marks, "data": "synthetic (seeded; workload.py)", "studies": {}}
+    t0 = time.perf_counter()
+    for study, spec in LIFETIME_STUDIES.items():
+        base = W.CONFIGS[spec["base"]]
+        cfg = dataclasses.replace(base, name=f"{base.name}-lifetime-{study}", requests=spec["requests"],
+                                  heads=spec["heads"], pool_slots=spec["requests"], permute_slots=False,
+                                  steps=steps)
+        d, H, R = cfg.d, cfg.heads, cfg.requests
+        slots = torch.arange(R, dtype=torch.int32, device="cuda")
+        pin = W.make_plan(cfg)
+        X0 = torch.from_numpy(W.initial_state(cfg)).cuda()
+        S32 = X0.clone()
+        arms = {}
+        for name in ("uniform6", "stepquant", "calibrated"):
+            mode, p = mode_plan(cfg, name)
+            plan = S.stepq_plan_create(d, d, H, cfg.gate_kind, cfg.unit_kind, mode, p.bits, p.w)
+            sb = S.stepq_plan_slot_bytes(plan)
+            pool = S.stepq_pool_alloc(plan, R, torch.zeros(R * sb, dtype=torch.uint8, device="cuda"))
+            S.stepq_pack(plan, pool, slots, X0)
+            arms[name] = {"plan": plan, "pool": pool, "bits": p.bits,
+                          "ws": torch.empty(S.stepq_workspace_bytes(plan, R), dtype=torch.uint8, device="cuda"),
+                          "y": torch.empty((R, H, d), dtype=torch.float32, device="cuda"),
+                          "err": []}
+        del X0
+        y32 = torch.empty((R, H, d), dtype=torch.float32, device="cuda")
+        Sq = torch.empty((R, H, d, d), dtype=torch.float32, device="cuda")
+        dt = torch.bfloat16 if cfg.bf16_inputs else torch.float32
+        for step in range(steps):
+            si = W.step_inputs(cfg, step, pin)
+            q, k, v = (torch.from_numpy(a).to(dt).cuda() for a in (si.q, si.k, si.v))
+            beta, gate = torch.from_numpy(si.beta).cuda(), torch.from_numpy(si.gate).cuda()
+            S.stepq_fp32_step(S32, slots, q, k, v, beta, gate, y32, cfg.gate_kind)
+            for a in arms.values():
+                S.stepq_decode_step(a["plan"], a["pool"], slots, q, k, v, beta, gate, a["y"], a["ws"])
+            if step + 1 in marks:
+                for a in arms.values():
+                    S.stepq_unpack(a["plan"], a["pool"], slots, Sq)
+                    if cfg.unit_kind == W.UNIT_ROW:       # per key row: [R, H, d] -> [H * d]
+                        e = (Sq - S32).norm(dim=3) / S32.norm(dim=3).clamp_min(1e-30)
+                    else:                                  # per head: [R, H] -> [H]
+                        e = (Sq - S32).flatten(2).norm(dim=2) / S32.flatten(2).norm(dim=2).clamp_min(1e-30)
+                    a["err"].append(e.mean(dim=0).reshape(-1).double().cpu().numpy())
+        torch.cuda.synchronize()
+        half_life = np.asarray(pin.half_life, np.float64).reshape(-1)
+        res = {"units": "key rows" if cfg.unit_kind == W.UNIT_ROW else "heads", "n_units": int(half_life.size),
+               "workload": f"{R} requests x {H} heads, d_k=d_v={d}, "
+                           f"{'per-key-row' if cfg.gate_kind else 'per-head'} gates, half-lives log-uniform "
+                           f"in [1, {cfg.half_life_max:.0f}]", "arms": {}}
+        for name, a in arms.items():
+            errs = np.stack(a["err"])                       # [checkpoints, units]
+            acc = errs.mean(axis=0)
+            bits = np.asarray(a["bits"]).reshape(-1)
+            res["arms"][name] = {
+                "spearman_rho_accumulated": spearman_rho(half_life, acc),
+                "spearman_rho_final": spearman_rho(half_life, errs[-1]),
+                "mean_error_accumulated": float(acc.mean()),
+                "mean_error_final": float(errs[-1].mean()),
+                "units_by_bits": {int(b): int(np.sum(bits == b)) for b in (4, 6, 8, 16) if np.sum(bits == b)},
+                "device_status": S.stepq_get_status(a["pool"])}
+        out["studies"][study] = res
+    out["seconds"] = time.perf_counter() - t0
+    if dist.rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 PIPE_HIDDEN = 5120          # model width of the projection proxy (a 27B-class hybrid model)
 
 
@@ -837,6 +981,50 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+SUB_CONFIGS = [("kda", "stepquant"), ("pool", "stepquant"), ("pool", "uniform8"), ("rollout", "stepquant")]
+
+
+def measure_config(name, mode, steps, kernel_steps, warmup, hbm_peak, alu_peak, dist):
+    """One more workload at full size on this GPU: plain decode steps between
+    two events (as the headline), each kernel alone, the fp32-state step."""
+    import torch
+    cfg = W.CONFIGS[name]
+    wl = DeviceWorkload(cfg, mode)
+
+    for s in range(warmup):
+        wl.run_step(s)
+    wl.join()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(wl.main)
+    for s in range(steps):
+        wl.run_step(warmup + s)
+    wl.join()
+    b.record(wl.main)
+    torch.cuda.synchronize()
+    ms = dist.max(a.elapsed_time(b)) / steps
+    rd_ms, fit_ms = time_isolated(wl, kernel_steps, warmup)
+    alg = algorithmic_bytes(cfg, wl.pin, wl.head_bytes)
+    rd_bytes = readout_bytes(cfg, wl.head_bytes)
+    ops = fit_alu_ops(cfg, wl.pin, wl.mode)
+    fp32 = time_fp32(cfg, wl.pin, kernel_steps, warmup)
+    out = {"workload": workload_config(cfg, mode, wl)["workload"], "quantizer": mode,
+           "value": dist.world * cfg.requests * cfg.heads / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+           "steps": steps, "hbm_gbs": dist.world * alg / (ms * 1e-3) / 1e9,
+           "hbm_frac": alg / (ms * 1e-3) / 1e9 / hbm_peak, "bytes_per_step": alg,
+           "slot_bytes": wl.slot_bytes, "compression_vs_fp32": W.fp32_state_bytes(cfg) / wl.slot_bytes,
+           "readout": {"us_alone": rd_ms * 1e3, "gbs_alone": rd_bytes / (rd_ms * 1e-3) / 1e9,
+                       "frac_hbm_alone": rd_bytes / (rd_ms * 1e-3) / 1e9 / hbm_peak},
+           "fitpack": {"us_alone": fit_ms * 1e3, "fp32_ops": ops,
+                       "frac_alu_alone": ops / (fit_ms * 1e-3) / 1e12 / alu_peak},
+           "fp32_state_baseline": fp32}
+    if fp32 is not None:
+        fp32["frac_hbm"] = fp32["hbm_gbs"] / hbm_peak
+    del wl
+    torch.cuda.empty_cache()
+    return out
+
+
 def workload_config(cfg, mode, wl):
     pin = wl.pin if wl is not None else mode_plan(cfg, mode)[1]
     counts = {int(b): int(np.sum(pin.bits == b)) for b in (4, 6, 8, 16) if np.sum(pin.bits == b)}
@@ -889,10 +1077,10 @@ def main():
             run_reference(args)
         return
     dist = Dist(args.gpus)
-    if args.drift or args.pipeline:
+    if args.drift or args.pipeline or args.lifetime_study:
         import torch
         torch.cuda.set_device(dist.local)
-        (run_drift if args.drift else run_pipeline)(args, dist)
+        (run_lifetime_study if args.lifetime_study else run_drift if args.drift else run_pipeline)(args, dist)
         dist.close()
         return
     import torch
@@ -911,7 +1099,8 @@ def main():
     wl = DeviceWorkload(cfg, args.mode)
     cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
     gpu_index = cvd.split(",")[dist.local].strip() if cvd else str(dist.local)
-    ms, readout_ms, fit_ms, clocks = time_device(wl, args.steps, args.warmup, dist, gpu_index)
+    ms, clocks = time_device(wl, args.steps, args.warmup, dist, gpu_index)
+    readout_ms, fit_ms = time_kernels_overlapped(wl, args.kernel_steps, args.warmup)
     # which kernel bounds the step: each kernel timed alone (the overlapped
     # durations above share the SMs with the other stream)
     iso_readout_ms, iso_fit_ms = time_isolated(wl, args.isolated_steps, args.warmup)
@@ -935,9 +1124,11 @@ def main():
             "fitpack": {"us": fit_ms * 1e3, "fp32_ops": ops, "tops": fit_tops, "frac_alu": fit_tops / alu_peak,
                         "us_alone": iso_fit_ms * 1e3, "tops_alone": iso_fit_tops,
                         "frac_alu_alone": iso_fit_tops / alu_peak},
-            "note": "us: average launch duration inside the timed region, where the two streams overlap "
-                    f"and share the SMs; us_alone: the kernel alone on one stream ({args.isolated_steps} steps "
-                    "after the timed region); the roofline kernel is the one with the longer us_alone"}
+            "note": f"us: average launch duration in a separate pass of {args.kernel_steps} overlapped steps "
+                    "(the split calls with events on each kernel's stream; the two streams share the SMs); "
+                    f"us_alone: the kernel alone on one stream ({args.isolated_steps} steps); the headline "
+                    "timed region runs plain stepq_decode_step calls only; the roofline kernel is the one "
+                    "with the longer us_alone"}
     if iso_fit_ms >= iso_readout_ms:
         roof = {"kernel": "fitpack (k_quant, fit+pack)", "bound": "alu", "achieved": fit_tops,
                 "peak": alu_peak, "unit": "T fp32 lane-ops/s", "frac": fit_tops / alu_peak,
@@ -965,6 +1156,17 @@ def main():
         fp32["frac_hbm"] = fp32["hbm_gbs"] / hbm_peak
         fp32["value"] *= dist.world
 
+    config_obj = workload_config(cfg, args.mode, wl)
+    configs = {}
+    if args.config_steps > 0 and args.config == "gdn" and args.mode == "stepquant":
+        del wl
+        torch.cuda.empty_cache()
+        for name, mode in SUB_CONFIGS:
+            key = name if mode == "stepquant" else f"{name}_{mode}"
+            configs[key] = measure_config(name, mode, args.config_steps, min(args.config_steps, 100),
+                                          10, hbm_peak, alu_peak, dist)
+        wl = None
+
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
         orc = OracleRunner(cfg, args.mode)
@@ -981,11 +1183,12 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded; workload.py)",
-                "config": workload_config(cfg, args.mode, wl),
+                "config": config_obj,
                 "hbm_gbs": hbm_gbs, "hbm_frac": hbm_gbs / hbm_peak, "hbm_peak_gbs": hbm_peak,
                 "hbm_peak_source": peak_src, "bytes_per_step": alg_bytes,
                 "roofline": roof, "kernels": kern,
                 "fp32_state_baseline": fp32,
+                "configs": configs or None,
                 "serial_step": serial,
                 "graph": graph,
                 "cpu_baseline": cpu,

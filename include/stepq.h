@@ -211,6 +211,11 @@ STEPQ_API int stepq_decode_fitpack(const stepq_plan *plan, stepq_pool *pool,
  * previous step's fit on this pool, so back-to-back steps are safe.  With
  * side_stream == main_stream (or NULL) both halves run on main_stream.
  * Arguments as for the two halves.  Slots must be distinct within one call.
+ * A batch whose packed state exceeds 48 MB is stepped in chunks of requests
+ * (a multiple of 16 each): chunk by chunk, the readout on main_stream, an
+ * event, that chunk's fit + pack on side_stream -- so the fit re-reads the
+ * slots while they are still in L2 and the next chunk's readout overlaps it.
+ * The results are those of one launch of each half.
  * The fit still reads k, gate and workspace after the call returns: do not
  * overwrite them, or hand the same workspace to another pool's step, until
  * side_stream has finished this step (one workspace per layer in flight).
@@ -266,8 +271,11 @@ STEPQ_API int stepq_fp32_step(int32_t d_k, int32_t d_v, int32_t n_heads, int32_t
  * GPU that loads the library, held until the process exits.
  *   - n * n_heads * d_v must not exceed STEPQ_STATIC_DELTA_FLOATS, else
  *     STEPQ_ERR_INVALID and nothing is launched.
- *   - the first call on a device looks up the array's device address once
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and keeps it for that device's current context;
+ *     a call after the context changed (e.g. after cudaDeviceReset) looks it
+ *     up again.  Make the first call on a device, and the first after a
+ *     reset, before any stream capture.
  *   - every call shares the one array: calls whose kernels can overlap on the
  *     GPU (another stream, or the fit of the previous call on side_stream
  *     still running when the next call's readout starts on a different pool)
@@ -307,6 +315,19 @@ STEPQ_API int stepq_decode_step_static(const stepq_plan *plan, stepq_pool *pool,
 STEPQ_API int stepq_unit_distortion(const stepq_plan *plan, stepq_pool *pool,
                                     const int32_t *slot_idx, int64_t n, const float *X,
                                     double *dist, void *stream);
+
+/* The same distortion summed over the n requests and added on the device to
+ * dist_sum (the calibration total over all calibration states; hyper.ai
+ * summary, Method, the Lifetime-Aware Bit Allocation paragraph):
+ * dist_sum[u] += sum_r (X[r] - S[r])^2 over unit u's entries.
+ *   dist_sum  device, float64 [units] (caller-owned, read and written;
+ *             zero it before the first call of a calibration)
+ * Other arguments as for stepq_unit_distortion.  The order in which the
+ * requests' contributions are added is not fixed (double-precision atomic
+ * adds), so repeated runs may differ in the last bits. */
+STEPQ_API int stepq_unit_distortion_accumulate(const stepq_plan *plan, stepq_pool *pool,
+                                               const int32_t *slot_idx, int64_t n, const float *X,
+                                               double *dist_sum, void *stream);
 
 /* Lifetime weight of each unit from its retention gates over calibration
  * steps: ell_u = mean of log(g) over the unit's gates and the steps, the error
@@ -376,6 +397,25 @@ STEPQ_API int stepq_get_status(stepq_pool *pool, uint32_t *out);
 
 /* Reset the pool's status word to 0, in stream order. */
 STEPQ_API int stepq_clear_status(stepq_pool *pool, void *stream);
+
+/*
+ * Failure-detection test hook (not a step of the paper's method).  Every
+ * device wait of the library is bounded: a kernel that waits on a
+ * bulk-async copy gives up after a time limit, records STEPQ_DEV_TIMEOUT in
+ * the pool's status word and skips that head, leaving the GPU usable.  To
+ * let a test make such a wait run out without any fault, this call switches
+ * the readout and fit kernels of this pool's later calls to a mode in which
+ * they issue no staging copy at all (nothing is in flight) and wait at most
+ * wait_limit_us microseconds per wait; their heads are then skipped: y,
+ * the workspace and the pool's slots are left as they were.
+ *   flags         STEPQ_TEST_NO_STAGING_COPY, or 0 to restore normal
+ *                 operation (the default limit, 2 s).
+ *   wait_limit_us 1 .. 1000000 when flags != 0.
+ * STEPQ_ERR_INVALID on bad arguments.  Host-only; takes effect for calls
+ * made after it returns.
+ */
+#define STEPQ_TEST_NO_STAGING_COPY 1u
+STEPQ_API int stepq_pool_set_test_faults(stepq_pool *pool, uint32_t flags, uint32_t wait_limit_us);
 
 /* Message for the last failing call on this thread ("" if none). */
 STEPQ_API const char *stepq_last_error(void);

@@ -59,6 +59,7 @@ def lib():
         L.orc_quantize_head.argtypes = [P, I, P, P, P, P, P]
         L.orc_quantize_head.restype = I
         L.orc_delta_update.argtypes = [I, I, P, P, P, P, F, P, I, P, P]
+        L.orc_delta_update_d.argtypes = [I, I, P, P, P, P, F, P, I, P, P, P]
         L.orc_step_head.argtypes = [P, I, P, P, P, P, F, P, P, P]
         L.orc_step_head.restype = I
         L.orc_pack.argtypes = [P, P, I64, P, I64, P]
@@ -211,15 +212,17 @@ class Plan:
         return y, st
 
 
-def delta_update(S, q, k, v, beta, gate, gate_kind):
-    """X = D S + beta k (v^T - k^T D S) and y = X^T q on one head (float32)."""
+def delta_update(S, q, k, v, beta, gate, gate_kind, with_delta=False):
+    """X = D S + beta k (v^T - k^T D S) and y = X^T q on one head (float32);
+    with ``with_delta`` also delta = beta (v - k^T D S) [dv]."""
     S = _f32(S)
     dk, dv = S.shape
     X = np.zeros((dk, dv), np.float32)
     y = np.zeros(dv, np.float32)
-    lib().orc_delta_update(dk, dv, _p(S), _p(_f32(q)), _p(_f32(k)), _p(_f32(v)), float(beta),
-                           _p(_f32(np.atleast_1d(gate))), int(gate_kind), _p(X), _p(y))
-    return X, y
+    delta = np.zeros(dv, np.float32)
+    lib().orc_delta_update_d(dk, dv, _p(S), _p(_f32(q)), _p(_f32(k)), _p(_f32(v)), float(beta),
+                             _p(_f32(np.atleast_1d(gate))), int(gate_kind), _p(X), _p(y), _p(delta))
+    return (X, y, delta) if with_delta else (X, y)
 
 
 def fp32_step(S, slot_idx, q, k, v, beta, gate, gate_kind):

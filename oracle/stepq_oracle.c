@@ -549,9 +549,10 @@ int orc_quantize_head(const void *p, int h, const float *X, uint8_t *blob,
 /* evaluated by numpy in float64.                                            */
 /* ------------------------------------------------------------------------ */
 
-void orc_delta_update(int dk, int dv, const float *S, const float *q, const float *k,
-                      const float *v, float beta, const float *gate, int gate_kind,
-                      float *X, float *y)
+/* As orc_delta_update, also storing delta [dv] when delta_out is not NULL. */
+void orc_delta_update_d(int dk, int dv, const float *S, const float *q, const float *k,
+                        const float *v, float beta, const float *gate, int gate_kind,
+                        float *X, float *y, float *delta_out)
 {
     int i, j;
     for (j = 0; j < dv; j++) {
@@ -561,6 +562,8 @@ void orc_delta_update(int dk, int dv, const float *S, const float *q, const floa
             u = u + k[i] * (g * S[i * dv + j]);   /* (k^T D S)_j */
         }
         delta = beta * (v[j] - u);
+        if (delta_out)
+            delta_out[j] = delta;
         for (i = 0; i < dk; i++) {
             float g = gate_kind ? gate[i] : gate[0];
             X[i * dv + j] = g * S[i * dv + j] + k[i] * delta;
@@ -572,6 +575,13 @@ void orc_delta_update(int dk, int dv, const float *S, const float *q, const floa
             acc = acc + q[i] * X[i * dv + j];     /* (X^T q)_j */
         y[j] = acc;
     }
+}
+
+void orc_delta_update(int dk, int dv, const float *S, const float *q, const float *k,
+                      const float *v, float beta, const float *gate, int gate_kind,
+                      float *X, float *y)
+{
+    orc_delta_update_d(dk, dv, S, q, k, v, beta, gate, gate_kind, X, y, NULL);
 }
 
 /* One quantised decode step of one head in place on its blob. */

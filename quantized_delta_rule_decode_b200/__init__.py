@@ -18,6 +18,7 @@ from ._ffi import (  # noqa: F401
     GATE_SCALAR,
     MODE_STEPQUANT,
     MODE_UNIFORM,
+    TEST_NO_STAGING_COPY,
     UNIT_HEAD,
     UNIT_ROW,
     Plan,
@@ -43,9 +44,11 @@ from ._ffi import (  # noqa: F401
     stepq_plan_head_layout,
     stepq_row_impact,
     stepq_unit_distortion,
+    stepq_unit_distortion_accumulate,
     stepq_plan_slot_bytes,
     stepq_pool_alloc,
     stepq_pool_free,
+    stepq_pool_set_test_faults,
     stepq_unpack,
     stepq_workspace_bytes,
 )

@@ -12,6 +12,7 @@ _LIB_PATH = os.path.join(_HERE, "libstepq.so")
 
 OK, ERR_INVALID, ERR_CUDA, ERR_UNSUPPORTED = 0, 1, 2, 3
 DEV_BAD_SLOT, DEV_NONFINITE, DEV_TIMEOUT = 1, 2, 4
+TEST_NO_STAGING_COPY = 1
 GATE_SCALAR, GATE_DIAG = 0, 1
 UNIT_HEAD, UNIT_ROW = 0, 1
 MODE_STEPQUANT, MODE_UNIFORM = 0, 1
@@ -38,12 +39,14 @@ _SIGS = {
     "stepq_decode_step_host": [_P, _P, _P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P],
     "stepq_decode_step_static": [_P, _P, _P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P, _P],
     "stepq_unit_distortion": [_P, _P, _P, _I64, _P, _P, _P],
+    "stepq_unit_distortion_accumulate": [_P, _P, _P, _I64, _P, _P, _P],
     "stepq_lifetime_weight": [_I64, _I64, _I32, _P, _P],
     "stepq_allocate_bits": [_I64, _P, _P, _I32, _I64, _P],
     "stepq_row_impact": [_I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P],
     "stepq_impact_weights": [_I64, _I64, _P, _P],
     "stepq_get_status": [_P, ctypes.POINTER(ctypes.c_uint32)],
     "stepq_clear_status": [_P, _P],
+    "stepq_pool_set_test_faults": [_P, ctypes.c_uint32, ctypes.c_uint32],
     "stepq_last_error": [],
 }
 
@@ -308,6 +311,16 @@ def stepq_unit_distortion(plan: Plan, pool: Pool, slot_idx, X, dist=None, stream
     return dist
 
 
+def stepq_unit_distortion_accumulate(plan: Plan, pool: Pool, slot_idx, X, dist_sum, stream=None):
+    """dist_sum [units] (float64, on the device) += the per-unit squared
+    reconstruction error summed over the requests."""
+    import torch
+    s, n = _slots(slot_idx)
+    _call("stepq_unit_distortion_accumulate", plan.handle, pool.handle, s, n,
+          _ptr(X, torch.float32, "X"), _ptr(dist_sum, torch.float64, "dist_sum"), _stream(stream))
+    return dist_sum
+
+
 def stepq_lifetime_weight(gate) -> np.ndarray:
     """gate: host float32 [n_steps][n_units][gates_per_unit] (or [n_steps][n_units])."""
     g = np.ascontiguousarray(gate, np.float32)
@@ -357,3 +370,10 @@ def stepq_get_status(pool: Pool) -> int:
 
 def stepq_clear_status(pool: Pool, stream=None):
     _call("stepq_clear_status", pool.handle, _stream(stream))
+
+
+def stepq_pool_set_test_faults(pool: Pool, flags: int, wait_limit_us: int = 0):
+    """Test hook: with TEST_NO_STAGING_COPY the pool's readout and fit kernels
+    issue no staging copy and give up each wait after wait_limit_us (0 flags:
+    normal operation)."""
+    _call("stepq_pool_set_test_faults", pool.handle, int(flags), int(wait_limit_us))

@@ -28,7 +28,7 @@ import numpy as np
 
 from ._ffi import (MODE_STEPQUANT, UNIT_ROW, stepq_allocate_bits, stepq_impact_weights,
                    stepq_lifetime_weight, stepq_pack, stepq_plan_create, stepq_pool_alloc,
-                   stepq_plan_slot_bytes, stepq_row_impact, stepq_unit_distortion)
+                   stepq_plan_slot_bytes, stepq_row_impact, stepq_unit_distortion_accumulate)
 
 WIDTHS = (4, 6, 8)
 
@@ -59,8 +59,8 @@ def measure_distortion(d_k, d_v, n_heads, gate_kind, unit_kind, w, states, strea
 
     states: device fp32 tensors [n][n_heads][d_k][d_v] (any n per tensor).
     Returns float64 [units][3]: per unit, the squared reconstruction error
-    summed over the states in the given order and, within one, over the
-    requests in ascending order."""
+    summed over every request of every state tensor, on the device
+    (stepq_unit_distortion_accumulate); this function only passes buffers."""
     import torch
     units = n_heads * d_k if unit_kind == UNIT_ROW else n_heads
     total = np.zeros((units, 3), np.float64)
@@ -68,15 +68,18 @@ def measure_distortion(d_k, d_v, n_heads, gate_kind, unit_kind, w, states, strea
         plan = stepq_plan_create(d_k, d_v, n_heads, gate_kind, unit_kind, MODE_STEPQUANT,
                                  np.full(units, b, np.uint8), w)
         sb = stepq_plan_slot_bytes(plan)
+        dist_sum = None
         for X in states:
             n = X.shape[0]
+            if dist_sum is None:
+                dist_sum = torch.zeros(units, dtype=torch.float64, device=X.device)
             buf = torch.zeros(n * sb, dtype=torch.uint8, device=X.device)
             pool = stepq_pool_alloc(plan, n, buf)
             slots = torch.arange(n, dtype=torch.int32, device=X.device)
             stepq_pack(plan, pool, slots, X, stream=stream)
-            dist = stepq_unit_distortion(plan, pool, slots, X, stream=stream).cpu().numpy()
-            for r in range(n):
-                total[:, col] += dist[r]
+            stepq_unit_distortion_accumulate(plan, pool, slots, X, dist_sum, stream=stream)
+        if dist_sum is not None:
+            total[:, col] = dist_sum.cpu().numpy()
     return total
 
 

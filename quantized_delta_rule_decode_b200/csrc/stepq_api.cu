@@ -22,6 +22,7 @@ struct stepq_plan {
     std::vector<uint16_t> row_off;
     std::vector<float> w, kappa, qmax_hi;
     std::vector<int16_t> qheads, pheads;
+    std::vector<uint8_t> chunk_rows;
     uint32_t max_qhead_bytes = 0;
     void *dev_tables = nullptr;
     stepq::PlanDev dev{};
@@ -36,6 +37,8 @@ struct stepq_pool {
     cudaEvent_t readout_done = nullptr;
     cudaEvent_t fit_done = nullptr;
     bool fit_pending = false;
+    uint32_t test_faults = 0;
+    uint64_t wait_limit_ns = stepq::kDefaultWaitLimitNs;
 };
 
 namespace {
@@ -98,6 +101,8 @@ stepq::StepArgs base_args(const stepq_plan *plan, stepq_pool *pool, const int32_
     a.slot_idx = slot_idx;
     a.n = n;
     a.status = pool->status;
+    a.test_faults = pool->test_faults;
+    a.wait_limit_ns = pool->wait_limit_ns;
     (void)plan;
     return a;
 }
@@ -156,6 +161,7 @@ int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out) {
     p->row_bits.resize((size_t)H * dk); p->row_off.resize((size_t)H * dk);
     p->w.assign(d.w, d.w + (size_t)H * dk);
     p->kappa.resize((size_t)H * dk);
+    p->chunk_rows.resize(H);
     size_t off = 0;
     for (int h = 0; h < H; ++h) {
         bool all_same = true, any_pivot = false;
@@ -181,6 +187,12 @@ int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out) {
                 b == 16 ? 0.0f : (float)qhi / (float)((1 << (b - 1)) - 1);
         }
         p->scale_off[h] = (uint32_t)hb;
+        int widest = 0;
+        for (int i = 0; i < dk; ++i) {
+            const int b = p->row_bits[(size_t)h * dk + i];
+            widest = std::max(widest, b == 16 ? 2 * dv : dv * b / 8);
+        }
+        p->chunk_rows[h] = (uint8_t)stepq::readout_chunk_rows(dk, widest);
         if (pivot_head) {
             p->pheads.push_back((int16_t)h);
         } else {
@@ -207,7 +219,8 @@ int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out) {
     size_t o_roff = round_up(o_rbits + HD, 16), o_w = round_up(o_roff + 2 * HD, 16);
     size_t o_kap = o_w + 4 * HD, o_qhi = o_kap + 4 * HD;
     size_t o_qh = round_up(o_qhi + 4 * H, 16), o_ph = round_up(o_qh + 2 * H, 16);
-    size_t total = o_ph + 2 * H;
+    size_t o_chunk = round_up(o_ph + 2 * H, 16);
+    size_t total = o_chunk + H;
     std::vector<uint8_t> host(total, 0);
     memcpy(&host[o_head_off], p->head_off.data(), 4 * H);
     memcpy(&host[o_head_bytes], p->head_bytes.data(), 4 * H);
@@ -221,6 +234,7 @@ int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out) {
     memcpy(&host[o_qhi], p->qmax_hi.data(), 4 * H);
     if (!p->qheads.empty()) memcpy(&host[o_qh], p->qheads.data(), 2 * p->qheads.size());
     if (!p->pheads.empty()) memcpy(&host[o_ph], p->pheads.data(), 2 * p->pheads.size());
+    memcpy(&host[o_chunk], p->chunk_rows.data(), H);
     cudaError_t e = cudaGetDevice(&p->device);
     if (e == cudaSuccess) e = cudaMalloc(&p->dev_tables, total);
     if (e == cudaSuccess) e = cudaMemcpy(p->dev_tables, host.data(), total, cudaMemcpyHostToDevice);
@@ -250,6 +264,7 @@ int stepq_plan_create(const stepq_plan_desc *desc, stepq_plan **out) {
     v.max_qhead_bytes = p->max_qhead_bytes;
     v.qheads = reinterpret_cast<const int16_t *>(t + o_qh);
     v.pheads = reinterpret_cast<const int16_t *>(t + o_ph);
+    v.chunk_rows = t + o_chunk;
     *out = p;
     return STEPQ_OK;
 }
@@ -360,8 +375,21 @@ int stepq_unpack(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_i
     return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "unpack launch");
 }
 
+static int unit_distortion(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_idx,
+                           int64_t n, const float *X, double *dist, void *stream, bool accumulate);
+
 int stepq_unit_distortion(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_idx,
                           int64_t n, const float *X, double *dist, void *stream) {
+    return unit_distortion(plan, pool, slot_idx, n, X, dist, stream, false);
+}
+
+int stepq_unit_distortion_accumulate(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_idx,
+                                     int64_t n, const float *X, double *dist_sum, void *stream) {
+    return unit_distortion(plan, pool, slot_idx, n, X, dist_sum, stream, true);
+}
+
+static int unit_distortion(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_idx,
+                           int64_t n, const float *X, double *dist, void *stream, bool accumulate) {
     g_err.clear();
     int rc = check_pool(plan, pool);
     if (!rc) rc = check_rows(plan, slot_idx, n);
@@ -373,6 +401,7 @@ int stepq_unit_distortion(const stepq_plan *plan, stepq_pool *pool, const int32_
     stepq::StepArgs a = base_args(plan, pool, slot_idx, n);
     a.X = X;
     a.dist = dist;
+    a.dist_accumulate = accumulate ? 1 : 0;
     cudaError_t e = stepq::launch_distortion(plan->dev, a, s);
     return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "distortion launch");
 }
@@ -438,21 +467,63 @@ int stepq_decode_fitpack(const stepq_plan *plan, stepq_pool *pool, const int32_t
     return STEPQ_OK;
 }
 
+// A batch whose packed state is larger than a share of L2 is stepped in
+// chunks of requests: each chunk's readout (main stream) is followed, after
+// an event, by that chunk's fit + pack (side stream), so the fit re-reads the
+// blobs while the readout has just brought them into L2 and the next chunk's
+// readout overlaps it.  Every head is computed exactly as in one launch.
+constexpr size_t kChunkStateBytes = 48ull << 20;
+
 int stepq_decode_step(const stepq_plan *plan, stepq_pool *pool, const int32_t *slot_idx, int64_t n,
                       int32_t qkv_dtype, const void *q, const void *k, const void *v,
                       const float *beta, const float *gate, float *y, void *workspace,
                       size_t ws_bytes, void *main_stream, void *side_stream) {
-    int rc = stepq_decode_readout(plan, pool, slot_idx, n, qkv_dtype, q, k, v, beta, gate, y,
-                                  workspace, ws_bytes, main_stream);
-    if (rc || n == 0) return rc;
+    // the whole batch's arguments are checked (and the previous step's fit
+    // waited for) by the readout of the first chunk, called on all of them
+    g_err.clear();
+    int rc = check_pool(plan, pool);
+    if (!rc) rc = check_rows(plan, slot_idx, n);
+    if (rc) return rc;
+    if (n == 0) return STEPQ_OK;
+    if ((rc = check_step_inputs(plan, n, qkv_dtype, q, k, v, beta, gate, y, workspace, ws_bytes, true)))
+        return rc;
     cudaStream_t m = static_cast<cudaStream_t>(main_stream);
     cudaStream_t s = side_stream ? static_cast<cudaStream_t>(side_stream) : m;
-    if (s != m) {
-        cudaError_t e = cudaEventRecord(pool->readout_done, m);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, pool->readout_done, 0);
-        if (e != cudaSuccess) return cuda_fail(e, "stream handoff");
+    if ((rc = wait_pending_fit(pool, m))) return rc;
+    // requests per chunk: a multiple of 16 (every per-request input offset
+    // stays 16-byte aligned), chunks of near-equal size
+    int64_t most = std::max<int64_t>(16, (int64_t)(kChunkStateBytes / std::max<size_t>(plan->slot_bytes, 1)));
+    const int64_t nch = (n + most - 1) / most;
+    int64_t chunk = (n + nch - 1) / nch;
+    chunk = (chunk + 15) / 16 * 16;
+    const size_t H = (size_t)plan->H;
+    const size_t es = qkv_dtype == STEPQ_DTYPE_BF16 ? 2 : 4;
+    const size_t gate_per_req = plan->gate_kind == STEPQ_GATE_DIAG ? H * plan->dk : H;
+    for (int64_t r0 = 0; r0 < n; r0 += chunk) {
+        const int64_t nn = std::min(chunk, n - r0);
+        const uint8_t *qb = static_cast<const uint8_t *>(q), *kb = static_cast<const uint8_t *>(k);
+        const uint8_t *vb = static_cast<const uint8_t *>(v);
+        const size_t qkv_off = (size_t)r0 * H * plan->dk * es;
+        stepq::StepArgs a = base_args(plan, pool, slot_idx + r0, nn);
+        a.q = qb + qkv_off; a.k = kb + qkv_off; a.v = vb + qkv_off;
+        a.beta = beta + (size_t)r0 * H;
+        a.gate = gate + (size_t)r0 * gate_per_req;
+        a.y = y + (size_t)r0 * H * plan->dv;
+        a.delta = static_cast<float *>(workspace) + (size_t)r0 * H * plan->dv;
+        cudaError_t e = stepq::launch_readout(plan->dev, a, qkv_dtype, m);
+        if (e != cudaSuccess) return cuda_fail(e, "readout launch");
+        if (s != m) {
+            e = cudaEventRecord(pool->readout_done, m);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(s, pool->readout_done, 0);
+            if (e != cudaSuccess) return cuda_fail(e, "stream handoff");
+        }
+        e = stepq::launch_fitpack(plan->dev, a, qkv_dtype, s);
+        if (e != cudaSuccess) return cuda_fail(e, "fitpack launch");
     }
-    return stepq_decode_fitpack(plan, pool, slot_idx, n, qkv_dtype, k, gate, workspace, ws_bytes, s);
+    cudaError_t e = cudaEventRecord(pool->fit_done, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    pool->fit_pending = true;
+    return STEPQ_OK;
 }
 
 namespace {
@@ -585,6 +656,17 @@ int stepq_get_status(stepq_pool *pool, uint32_t *out) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess) e = cudaMemcpy(out, pool->status, 4, cudaMemcpyDeviceToHost);
     return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "status read");
+}
+
+int stepq_pool_set_test_faults(stepq_pool *pool, uint32_t flags, uint32_t wait_limit_us) {
+    g_err.clear();
+    if (!pool) return fail(STEPQ_ERR_INVALID, "pool is NULL");
+    if (flags & ~STEPQ_TEST_NO_STAGING_COPY) return fail(STEPQ_ERR_INVALID, "unknown test flags %#x", flags);
+    if (flags && (wait_limit_us < 1 || wait_limit_us > 1000000))
+        return fail(STEPQ_ERR_INVALID, "wait_limit_us %u outside 1 .. 1000000", wait_limit_us);
+    pool->test_faults = flags;
+    pool->wait_limit_ns = flags ? (uint64_t)wait_limit_us * 1000ull : stepq::kDefaultWaitLimitNs;
+    return STEPQ_OK;
 }
 
 int stepq_clear_status(stepq_pool *pool, void *stream) {

@@ -36,7 +36,17 @@ struct PlanDev {
     uint32_t max_qhead_bytes;    // largest blob of a quantised (non-pivot) head
     const int16_t *qheads;       // [n_qheads] indices of the quantised heads
     const int16_t *pheads;       // [n_pheads] indices of the FP16 pivot heads
+    const uint8_t *chunk_rows;   // [H] rows per staged chunk of the readout (readout_chunk_rows)
 };
+
+// The readout stages a head's packed rows into shared memory in chunks of
+// whole rows, at most 32 * d bytes each (4 KB at d = 128): the largest power
+// of two of rows, at most d, whose widest row fits that many times.
+__host__ __device__ constexpr int readout_chunk_rows(int d, int max_row_bytes) {
+    int r = d;
+    while (r > 1 && r * max_row_bytes > 32 * d) r >>= 1;
+    return r;
+}
 
 // Everything a decode / pack launch needs besides the plan.
 struct StepArgs {
@@ -51,9 +61,14 @@ struct StepArgs {
     float *delta;      // workspace [n][H][dv]
     const float *X;    // pack input [n][H][dk][dv]
     float *S_out;      // unpack output
-    double *dist;      // per-unit distortion output [n][units]
+    double *dist;      // per-unit distortion output [n][units], or [units] summed (dist_accumulate)
+    int dist_accumulate;
     uint32_t *status;
+    uint32_t test_faults;   // STEPQ_TEST_* bits (0 in normal operation)
+    uint64_t wait_limit_ns; // bound on each device wait
 };
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 
 // ---- launchers (stepq_kernels.cu) ------------------------------------------
 cudaError_t launch_readout(const PlanDev &P, const StepArgs &a, int qkv_dtype, cudaStream_t s);

@@ -162,6 +162,16 @@ def rel_l2(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
+def rel_l2_worst_head(a, b):
+    """The largest relative L2 error of any one head's readout (last axis =
+    d_v): one small-norm head cannot hide inside a batch-wide norm."""
+    a = np.asarray(a, np.float64).reshape(-1, np.shape(a)[-1])
+    b = np.asarray(b, np.float64).reshape(-1, np.shape(b)[-1])
+    num = np.linalg.norm(a - b, axis=1)
+    den = np.maximum(np.linalg.norm(b, axis=1), 1e-300)
+    return float(np.max(num / den))
+
+
 class StepDiff:
     """Accumulates full-step blob differences over many heads."""
 

@@ -43,6 +43,37 @@ def test_unit_distortion_matches_oracle(name, R):
     assert S.stepq_get_status(pool) == 0
 
 
+@pytest.mark.parametrize("name", ["gdn", "kda"])
+def test_unit_distortion_accumulates_on_device(name):
+    """dist_sum += the distortion summed over requests, over two calls: the
+    oracle's per-request values summed in float64 (rel 1e-11: the device
+    adds in another order)."""
+    import torch
+    cfg = W.CONFIGS[name]
+    pair = Pair(cfg)
+    S = lib()
+    R = 3
+    slots = W.slot_indices(cfg)[:R] if cfg.permute_slots else np.arange(R, dtype=np.int32)
+    nslots = cfg.pool_slots if cfg.permute_slots else R
+    units = cfg.units
+    total = torch.zeros(units, dtype=torch.float64, device="cuda")
+    want = np.zeros(units, np.float64)
+    for call in range(2):
+        X = W.initial_state(cfg, [call * R + r for r in range(R)])
+        pool = pair.gpu_pool(nslots)
+        Xd = dev(X)
+        S.stepq_pack(pair.gpu, pool, dev(slots), Xd)
+        S.stepq_unit_distortion_accumulate(pair.gpu, pool, dev(slots), Xd, total)
+        o = pair.ora.new_pool(nslots)
+        assert pair.ora.pack(o, slots, X) == 0
+        d, st = pair.ora.unit_distortion(o, slots, X)
+        assert st == 0
+        want += d.sum(axis=0)
+        assert S.stepq_get_status(pool) == 0
+    got = total.cpu().numpy()
+    assert np.allclose(got, want, rtol=1e-11, atol=0)
+
+
 def _gates(cfg, pin):
     g = np.asarray(pin.gate, np.float32)
     if cfg.unit_kind == W.UNIT_ROW:

@@ -14,7 +14,8 @@ import numpy as np
 import pytest
 
 import workload as W
-from gpu_harness import Pair, StepDiff, compare_pack, dev, lib, new_stats, pool_to_host, rel_l2
+from gpu_harness import (Pair, StepDiff, compare_pack, dev, lib, new_stats, pool_to_host, rel_l2,
+                         rel_l2_worst_head)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,5 +73,6 @@ def test_fullsize_sampled(name, samples):
         yos.append(yo)
         diff.add(pair, h, pair.head_blob(g1, slots_np[r], h), blob, None)
     assert rel_l2(np.array(ys), np.array(yos)) <= 1e-5
+    assert rel_l2_worst_head(np.array(ys), np.array(yos)) <= 1e-5
     diff.check(1e-3)
     assert S.stepq_get_status(pool) == 0

@@ -21,7 +21,7 @@ import pytest
 
 import workload as W
 from gpu_harness import (Pair, StepDiff, compare_pack, dev, lib, new_stats, pool_to_host, rel_l2,
-                         step_tensors)
+                         rel_l2_worst_head, step_tensors)
 
 pytestmark = pytest.mark.gpu
 
@@ -46,10 +46,10 @@ def _oracle_step(pair, pool_bytes, slots, si, rr, hh):
     return y
 
 
-def _run_case(name, mode=W.MODE_STEPQUANT, ub=None, R=None, steps=1, two_streams=True):
+def _run_case(name, mode=W.MODE_STEPQUANT, ub=None, R=None, steps=1, two_streams=True, pivots=True):
     import torch
     cfg = W.CONFIGS[name]
-    pair = Pair(cfg, mode=mode, uniform_bits=ub)
+    pair = Pair(cfg, mode=mode, uniform_bits=ub, pivots=pivots)
     S = lib()
     R = R or cfg.requests
     reqs = list(range(R))
@@ -75,6 +75,7 @@ def _run_case(name, mode=W.MODE_STEPQUANT, ub=None, R=None, steps=1, two_streams
         before = o.copy()
         yo = _oracle_step(pair, o, slots, si, rr, hh).reshape(R, cfg.heads, cfg.d)
         assert rel_l2(y.cpu().numpy(), yo) <= 1e-5
+        assert rel_l2_worst_head(y.cpu().numpy(), yo) <= 1e-5
         diff = StepDiff()
         for r in range(R):
             for h in range(cfg.heads):
@@ -123,6 +124,17 @@ def test_step_kda_temporal_only():
 def test_step_kda_spatial_only():
     """Ablation: the dual-axis fit on uniform 6-bit key rows, no pivots."""
     _run_case("kda", mode=W.MODE_STEPQUANT, ub=6, R=2, steps=2)
+
+
+def test_step_gdn_nopivot():
+    """Ablation: the plan's widths with its FP16 pivot head quantised instead."""
+    pair = _run_case("gdn", R=4, steps=2, pivots=False)
+    assert not np.any(pair.pin.bits == 16)
+
+
+def test_step_kda_nopivot():
+    pair = _run_case("kda", R=2, steps=2, pivots=False)
+    assert not np.any(pair.pin.bits == 16)
 
 
 def test_two_streams_equal_one_stream_and_split_calls():
@@ -186,3 +198,38 @@ def test_unit_gate_zero_beta_keeps_reconstruction():
     for h in range(cfg.heads):
         # identical X (= S_prev) on both sides -> the pack contract applies
         compare_pack(pair, h, pair.head_blob(g, 0, h), pair.head_blob(o2, 0, h), Sprev[0, h], stats)
+
+
+@pytest.mark.parametrize("name", ["kda", "pool"])
+def test_chunked_step_equals_one_launch_of_each_half(name):
+    """A batch larger than the chunk budget (kda: 106 MB of packed state, pool:
+    310 MB) is stepped chunk by chunk; its readout and state must be exactly
+    those of one readout launch and one fit launch over the whole batch."""
+    import torch
+    cfg = W.CONFIGS[name]
+    pair = Pair(cfg)
+    S = lib()
+    R = cfg.requests
+    slots = dev(W.slot_indices(cfg))
+    X = torch.randn((R, cfg.heads, cfg.d, cfg.d), dtype=torch.float32, device="cuda")
+    X *= torch.exp(torch.randn((R, cfg.heads, cfg.d, 1), device="cuda"))
+    si = W.step_inputs(cfg, 0, pair.pin)
+    t = step_tensors(cfg, si)
+    outs = []
+    for how in ("chunked", "whole"):
+        pool = pair.gpu_pool(cfg.pool_slots)
+        S.stepq_pack(pair.gpu, pool, slots, X)
+        ws = torch.empty(S.stepq_workspace_bytes(pair.gpu, R), dtype=torch.uint8, device="cuda")
+        y = torch.empty((R, cfg.heads, cfg.d), dtype=torch.float32, device="cuda")
+        if how == "chunked":
+            S.stepq_decode_step(pair.gpu, pool, slots, t["q"], t["k"], t["v"], t["beta"], t["gate"], y, ws,
+                                None, torch.cuda.Stream())
+        else:
+            S.stepq_decode_readout(pair.gpu, pool, slots, t["q"], t["k"], t["v"], t["beta"], t["gate"], y, ws)
+            S.stepq_decode_fitpack(pair.gpu, pool, slots, t["k"], t["gate"], ws)
+        torch.cuda.synchronize()
+        outs.append((y.cpu().numpy(), pool_to_host(pool)))
+        assert S.stepq_get_status(pool) == 0
+        del pool, ws, y
+    assert np.array_equal(outs[0][0], outs[1][0])
+    assert np.array_equal(outs[0][1], outs[1][1])
