@@ -158,6 +158,8 @@ def parse():
     ap.add_argument("--lifetime-study", action="store_true",
                     help="instead of the throughput line: per-unit accumulated error of quantised rollouts "
                          "vs the fp32 rollout, and its Spearman correlation with the unit's gate half-life")
+    ap.add_argument("--timeline", action="store_true",
+                    help="instead of the throughput line: start/end of each kernel of a few overlapped steps")
     ap.add_argument("--pipeline", action="store_true",
                     help="instead of the throughput line: per-token time of a layer stack with GEMM proxies")
     ap.add_argument("--drift-arms", default="stepquant,impact,allocated,calibrated,temporal,uniform8,uniform6",
@@ -861,6 +863,47 @@ def run_lifetime_study(args, dist):
         print(json.dumps(out), flush=True)
 
 
+def run_timeline(args, dist):
+    """Start and end of every kernel of a few overlapped decode steps, on one
+    clock: CUDA events recorded on each kernel's own stream around the split
+    calls (readout on the main stream, fit + pack on the side stream after an
+    event), all read as offsets from one event at the start.  Shows where
+    layer l's fit runs beside layer l + 1's readout (the schedule of the
+    hyper.ai summary, Method, last paragraph)."""
+    import torch
+    cfg = W.CONFIGS[args.config]
+    wl = DeviceWorkload(cfg, args.mode)
+    steps = max(2 * wl.layers, 6)
+    for s in range(args.warmup):
+        wl.run_step(s)
+    wl.join()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    t0.record(wl.main)
+    for s in range(steps):
+        wl.run_step_timed(args.warmup + s, evs[s])
+    wl.join()
+    torch.cuda.synchronize()
+    rows = []
+    for s, e in enumerate(evs):
+        rows.append({"step": s, "layer": (args.warmup + s) % wl.layers,
+                     "readout_us": [t0.elapsed_time(e[0]) * 1e3, t0.elapsed_time(e[1]) * 1e3],
+                     "fit_us": [t0.elapsed_time(e[2]) * 1e3, t0.elapsed_time(e[3]) * 1e3]})
+    overlap = 0.0
+    for a, b in zip(rows, rows[1:]):
+        lo = max(a["fit_us"][0], b["readout_us"][0])
+        hi = min(a["fit_us"][1], b["readout_us"][1])
+        overlap += max(0.0, hi - lo)
+    out = {"report": "kernel timeline of overlapped decode steps (CUDA events on each kernel's stream)",
+           "workload": workload_config(cfg, args.mode, wl)["workload"], "layers": wl.layers,
+           "rows": rows, "readout_inside_previous_fit_us_total": overlap,
+           "note": "a readout event pair brackets the call, which first waits for this layer's previous "
+                   "fit; the readout kernel itself starts when SM resources free up"}
+    if dist.rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 PIPE_HIDDEN = 5120          # model width of the projection proxy (a 27B-class hybrid model)
 
 
@@ -1077,10 +1120,11 @@ def main():
             run_reference(args)
         return
     dist = Dist(args.gpus)
-    if args.drift or args.pipeline or args.lifetime_study:
+    if args.drift or args.pipeline or args.lifetime_study or args.timeline:
         import torch
         torch.cuda.set_device(dist.local)
-        (run_lifetime_study if args.lifetime_study else run_drift if args.drift else run_pipeline)(args, dist)
+        (run_lifetime_study if args.lifetime_study else run_drift if args.drift else
+         run_timeline if args.timeline else run_pipeline)(args, dist)
         dist.close()
         return
     import torch
