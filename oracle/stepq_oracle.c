@@ -47,6 +47,11 @@
  *     reproduce exactly for multi-step rollouts to agree; likewise the column
  *     maximum max_i |X_ij / r_i| takes the quotient as |X_ij| times the
  *     correctly rounded 1/r_i (times qmax_hi/qmax_i for rows of other widths).
+ *     That order is itself pinned to the definition: oracle/definition.py
+ *     evaluates the whole requantisation in float64 with no order, and
+ *     tests/test_oracle_fullsize_fit.py holds this file's factors,
+ *     candidates, objectives, argmin and codes to it on full-size heads of
+ *     every workload (differences only within derived rounding bounds).
  *
  * Parity status of each function is stated in its comment ("pinned by ...").
  */
