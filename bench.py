@@ -47,6 +47,8 @@ if ROOT not in sys.path:
 import workload as W  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
+FIT_STREAMS = 0             # side streams the layers' fits take in turn (0: one per layer pool)
+MAIN_PRIORITY = -5          # readout stream priority (lower is higher; mapped into the device's range)
 SMS, FP32_LANES = 148, 128
 METRIC = "quantized state-step throughput (head-updates/s) and HBM GB/s vs B200 peak"
 UNIT = "head-updates/s"
@@ -151,6 +153,10 @@ def parse():
                     help="steps of each further workload measured into the line's 'configs' (0: none)")
     ap.add_argument("--isolated-steps", type=int, default=500,
                     help="steps of the per-kernel timing with each kernel alone")
+    ap.add_argument("--fit-streams", type=int, default=FIT_STREAMS,
+                    help="side streams the layers' fit + pack launches take in turn (0: one per layer pool)")
+    ap.add_argument("--main-priority", type=int, default=MAIN_PRIORITY,
+                    help="priority of the readout stream (0: the default stream priority)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="skip the CUDA-graph replay of the same steps")
     ap.add_argument("--drift", action="store_true",
@@ -301,7 +307,7 @@ def fit_alu_ops(cfg, pin, mode=W.MODE_STEPQUANT):
 
 
 class DeviceWorkload:
-    def __init__(self, cfg, mode):
+    def __init__(self, cfg, mode, fit_streams=None):
         import torch
 
         import quantized_delta_rule_decode_b200 as S
@@ -346,15 +352,24 @@ class DeviceWorkload:
         # layer l+1's readout runs
         self.ws = [torch.empty(S.stepq_workspace_bytes(self.plan, R), dtype=torch.uint8, device="cuda")
                    for _ in range(self.layers)]
-        self.main = torch.cuda.current_stream()
-        self.side = torch.cuda.Stream()
+        # The readout (the step's critical path: it produces y) runs on a
+        # high-priority stream, so that its CTAs take SMs ahead of the fits as
+        # soon as any retire; each layer's fit + pack runs on a side stream of
+        # its own (or one of `fit_streams` taken in turn), so that one layer's
+        # fit can start in the tail of the previous layer's.
+        fs = FIT_STREAMS if fit_streams is None else fit_streams
+        self.fit_streams = self.layers if fs <= 0 else min(fs, self.layers)
+        self.main = torch.cuda.Stream(priority=MAIN_PRIORITY) if MAIN_PRIORITY else torch.cuda.current_stream()
+        self.sides = [torch.cuda.Stream() for _ in range(self.fit_streams)]
+        self.side = self.sides[0]
         L = S.load_library()
         self.L = L
         P = ctypes.c_void_p
-        ms, ss = P(self.main.cuda_stream), P(self.side.cuda_stream)
+        ms = P(self.main.cuda_stream)
         sp = P(self.slots.data_ptr())
         self.step_args, self.read_args, self.fit_args = [], [], []
         for layer in range(self.layers):
+            ss = P(self.side_of_layer(layer).cuda_stream)
             wsp, wsb = P(self.ws[layer].data_ptr()), self.ws[layer].numel()
             for t in self.ring:
                 common = (self.plan.handle, self.pools[layer].handle, sp, R, self.dtype_code)
@@ -365,6 +380,12 @@ class DeviceWorkload:
                 self.read_args.append(common + io + (ms,))
                 self.fit_args.append(common + (P(t["k"].data_ptr()), P(t["gate"].data_ptr()),
                                                wsp, wsb, ss))
+
+    def side_of_layer(self, layer):
+        return self.sides[layer % len(self.sides)]
+
+    def side_of(self, step):
+        return self.side_of_layer(step % self.layers)
 
     def args_index(self, step):
         return (step % self.layers) * 16 + (step % 16)
@@ -381,14 +402,16 @@ class DeviceWorkload:
         if self.L.stepq_decode_readout(*self.read_args[i]):
             raise RuntimeError(self.L.stepq_last_error().decode())
         ev[1].record(self.main)
-        self.side.wait_event(ev[1])
-        ev[2].record(self.side)
+        side = self.side_of(step)
+        side.wait_event(ev[1])
+        ev[2].record(side)
         if self.L.stepq_decode_fitpack(*self.fit_args[i]):
             raise RuntimeError(self.L.stepq_last_error().decode())
-        ev[3].record(self.side)
+        ev[3].record(side)
 
     def join(self):
-        self.main.wait_stream(self.side)
+        for side in self.sides:
+            self.main.wait_stream(side)
 
 
 def time_device(wl, steps, warmup, dist, clocks_gpu):
@@ -432,9 +455,30 @@ def time_kernels_overlapped(wl, steps, warmup):
         wl.run_step_timed(warmup + s, evs[s])
     wl.join()
     torch.cuda.synchronize()
-    readout_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    fit_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    return statistics.mean(readout_ms), statistics.mean(fit_ms)
+    t0 = evs[0][0]
+    readout = [(t0.elapsed_time(e[0]), t0.elapsed_time(e[1])) for e in evs]
+    fit = [(t0.elapsed_time(e[2]), t0.elapsed_time(e[3])) for e in evs]
+    return busy_per_launch(readout), busy_per_launch(fit)
+
+
+def busy_per_launch(intervals):
+    """Time during which at least one of the launches was in flight, per
+    launch: the union of their [start, end] intervals divided by their number.
+    For launches that do not overlap this is their mean duration; for launches
+    that overlap (layers' fits on different side streams) it is the time the
+    kernel adds to the step per launch."""
+    if not intervals:
+        return 0.0
+    total, cur_lo, cur_hi = 0.0, None, None
+    for lo, hi in sorted(intervals):
+        if cur_hi is None or lo > cur_hi:
+            if cur_hi is not None:
+                total += cur_hi - cur_lo
+            cur_lo, cur_hi = lo, hi
+        else:
+            cur_hi = max(cur_hi, hi)
+    total += cur_hi - cur_lo
+    return total / len(intervals)
 
 
 def time_isolated(wl, steps, warmup):
@@ -472,7 +516,8 @@ def time_graph(wl, steps):
     S, L = wl.S, wl.L
     P = ctypes.c_void_p
     period = wl.layers * 16 // math.gcd(wl.layers, 16)
-    cs, ss = torch.cuda.Stream(), torch.cuda.Stream()
+    cs = torch.cuda.Stream(priority=MAIN_PRIORITY) if MAIN_PRIORITY else torch.cuda.Stream()
+    ss = [torch.cuda.Stream() for _ in range(wl.fit_streams)]
     pools = [S.stepq_pool_alloc(wl.plan, wl.nslots, p.buf) for p in wl.pools]
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
@@ -483,9 +528,10 @@ def time_graph(wl, steps):
             for s in range(period):
                 a = list(wl.step_args[wl.args_index(s)])
                 a[1] = pools[s % wl.layers].handle
-                a[-2], a[-1] = P(cs.cuda_stream), P(ss.cuda_stream)
+                a[-2], a[-1] = P(cs.cuda_stream), P(ss[(s % wl.layers) % len(ss)].cuda_stream)
                 rcs.append(L.stepq_decode_step(*a))
-            cs.wait_stream(ss)
+            for side in ss:
+                cs.wait_stream(side)
         finally:
             g.capture_end()
     if any(rcs):
@@ -555,7 +601,7 @@ def time_e2e(wl, steps, warmup):
                          P(t["q"].data_ptr()), P(t["k"].data_ptr()), P(t["v"].data_ptr()),
                          P(t["beta"].data_ptr()), P(t["gate"].data_ptr()), P(y.data_ptr()),
                          P(ws.data_ptr()), ws.numel(), P(wl.main.cuda_stream),
-                         P(wl.side.cuda_stream)))
+                         P(wl.side_of_layer(layer).cuda_stream)))
     for s in range(warmup):
         wl.L.stepq_decode_step_host(*args[wl.args_index(s)])
     wl.join()
@@ -960,19 +1006,23 @@ def run_pipeline(args, dist):
                                      y32, cfg.gate_kind)
             torch.matmul(o_in, w_out[l], out=x_out)
 
+    torch.cuda.synchronize()   # the tensors above were made on the default stream
     out = {}
     for variant in ("two_streams", "one_stream", "gemm_only", "fp32_state"):
-        for tok in range(args.warmup):
-            token(tok, variant)
-        wl.join()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(wl.main)
-        for tok in range(args.steps):
-            token(tok, variant)
-        wl.join()
-        b.record(wl.main)
-        torch.cuda.synchronize()
+        # the GEMMs run on the readout's stream, so each readout follows its
+        # layer's input projection as in a model
+        with torch.cuda.stream(wl.main):
+            for tok in range(args.warmup):
+                token(tok, variant)
+            wl.join()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(wl.main)
+            for tok in range(args.steps):
+                token(tok, variant)
+            wl.join()
+            b.record(wl.main)
+            torch.cuda.synchronize()
         out[variant] = dist.max(a.elapsed_time(b) / args.steps)
     gemm = out["gemm_only"]
     line = {"report": "per-token critical path of a layer stack (GEMM proxy + state step)",
@@ -1083,8 +1133,11 @@ def workload_config(cfg, mode, wl):
                   "layer_pools_cycled": wl.layers,
                   "l2": f"inputs larger than L2: {wl.layers} layer pools x "
                         f"{wl.nslots * wl.slot_bytes / 1e6:.1f} MB cycled, no flush",
-                  "streams": "readout on main stream, fit+pack on a side stream; "
-                             "a layer's fit overlaps the next layer's readout"})
+                  "streams": (f"readout on a high-priority main stream, each layer's fit+pack on "
+                              + ("its own side stream" if wl.fit_streams == wl.layers else
+                                 f"one of {wl.fit_streams} side streams in turn")
+                              + "; a layer's fit overlaps the next layer's readout and the tail of the "
+                                "previous layer's fit")})
     return c
 
 
@@ -1113,7 +1166,9 @@ def ncu_traffic(kernel, workload):
 
 
 def main():
+    global FIT_STREAMS, MAIN_PRIORITY
     args = parse()
+    FIT_STREAMS, MAIN_PRIORITY = args.fit_streams, args.main_priority
     if args.impl == "reference":
         # the oracle on the host: rank 0 alone, no process group and no GPU
         if int(os.environ.get("RANK", "0")) == 0:
@@ -1168,8 +1223,10 @@ def main():
             "fitpack": {"us": fit_ms * 1e3, "fp32_ops": ops, "tops": fit_tops, "frac_alu": fit_tops / alu_peak,
                         "us_alone": iso_fit_ms * 1e3, "tops_alone": iso_fit_tops,
                         "frac_alu_alone": iso_fit_tops / alu_peak},
-            "note": f"us: average launch duration in a separate pass of {args.kernel_steps} overlapped steps "
-                    "(the split calls with events on each kernel's stream; the two streams share the SMs); "
+            "note": f"us: the kernel's busy time per launch (the union of its launches' event intervals / "
+                    f"launches) in a separate pass of {args.kernel_steps} overlapped steps (the split calls with "
+                    "events on each kernel's stream; the streams share the SMs, and consecutive layers' fits "
+                    "on different side streams may overlap); "
                     f"us_alone: the kernel alone on one stream ({args.isolated_steps} steps); the headline "
                     "timed region runs plain stepq_decode_step calls only; the roofline kernel is the one "
                     "with the longer us_alone"}

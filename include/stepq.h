@@ -219,6 +219,11 @@ STEPQ_API int stepq_decode_fitpack(const stepq_plan *plan, stepq_pool *pool,
  * The fit still reads k, gate and workspace after the call returns: do not
  * overwrite them, or hand the same workspace to another pool's step, until
  * side_stream has finished this step (one workspace per layer in flight).
+ * Streams: the fits of different pools (layers) are independent, so a caller
+ * may give consecutive layers different side streams; one layer's fit then
+ * fills the SMs its predecessor's last CTAs leave idle.  A main_stream of
+ * higher priority than the side streams lets each readout (which produces y)
+ * take SMs ahead of pending fit CTAs.
  */
 STEPQ_API int stepq_decode_step(const stepq_plan *plan, stepq_pool *pool,
                                 const int32_t *slot_idx, int64_t n, int32_t qkv_dtype,

@@ -1,4 +1,5 @@
-"""The rank correlation bench.py reports for the lifetime study."""
+"""Statistics bench.py reports: the rank correlation of the lifetime study and
+the per-launch busy time of kernels whose launches may overlap."""
 
 import numpy as np
 
@@ -33,3 +34,18 @@ def test_spearman_matches_scipy():
         a = rng.integers(0, 30, 200).astype(float)   # many ties
         b = a + rng.normal(0, 10, 200)
         assert abs(bench.spearman_rho(a, b) - stats.spearmanr(a, b).statistic) < 1e-12
+
+
+def test_busy_per_launch_disjoint_is_the_mean_duration():
+    iv = [(0.0, 2.0), (5.0, 6.0), (10.0, 13.0)]
+    assert bench.busy_per_launch(iv) == 2.0
+
+
+def test_busy_per_launch_counts_overlap_once():
+    # [0, 4] and [3, 7] cover [0, 7]; [7, 9] touches it; [12, 13] stands alone:
+    # union 9 + 1 = 10 over 4 launches
+    iv = [(3.0, 7.0), (0.0, 4.0), (12.0, 13.0), (7.0, 9.0)]
+    assert bench.busy_per_launch(iv) == 2.5
+    # one launch inside another adds nothing
+    assert bench.busy_per_launch([(0.0, 10.0), (2.0, 3.0)]) == 5.0
+    assert bench.busy_per_launch([]) == 0.0

@@ -3,15 +3,17 @@
 The pages run the scale fit and pack write-back on a second CUDA stream,
 overlapped with the following computation (hyper.ai summary, Method, last
 paragraph; rcap.io post, the sentence after the pseudocode).  The benchmark
-does this over several layers: layer l's fit + pack runs on the side stream
-while layer l + 1's readout runs on the main stream, each layer with its own
-pool and workspace, and the next step's readout of a layer waits for that
-layer's previous fit.  This test runs that schedule on the full gdn workload
-(64 requests x 32 heads per layer, three layers, eight steps), alternating
-stepq_decode_step with the split calls (stepq_decode_readout, an event,
-stepq_decode_fitpack on the side stream) that the benchmark's instrumented
-pass uses.  After every step of every layer, a copy of the pool taken on the
-side stream and of y taken on the main stream (so the steps still overlap)
+does this over several layers: the readouts run on a high-priority main
+stream, and layer l's fit + pack on one of two side streams taken in turn, so
+that it runs beside layer l + 1's readout and beside the start of layer
+l + 1's fit; each layer has its own pool and workspace, and the next step's
+readout of a layer waits for that layer's previous fit.  This test runs that
+schedule on the full gdn workload (64 requests x 32 heads per layer, three
+layers, eight steps), alternating stepq_decode_step with the split calls
+(stepq_decode_readout, an event, stepq_decode_fitpack on the side stream)
+that the benchmark's instrumented pass uses.  After every step of every
+layer, a copy of the pool taken on that layer's side stream and of y taken
+on the main stream (so the steps still overlap)
 are compared on sampled (request, head) pairs with the oracle continuing
 from its own state: identical bytes, and y within relative L2 1e-5 per head.
 A race (a missing event, a shared workspace) would show as a difference.
@@ -49,8 +51,9 @@ def test_overlapped_layers_match_oracle():
     picks = [sorted({(int(rng.integers(R)), int(rng.integers(H))) for _ in range(SAMPLES)})
              for _ in range(LAYERS)]
     blobs = [{(r, h): pair.head_blob(g0, r, h).copy() for r, h in picks[l]} for l in range(LAYERS)]
-    main = torch.cuda.current_stream()
-    side = torch.cuda.Stream()
+    main = torch.cuda.Stream(priority=-5)
+    sides = [torch.cuda.Stream(), torch.cuda.Stream()]
+    main.wait_stream(torch.cuda.current_stream())   # the packs above
     keep, snaps = [], []
     dt = torch.bfloat16
     for s in range(STEPS):
@@ -59,6 +62,8 @@ def test_overlapped_layers_match_oracle():
             q, k, v = (torch.from_numpy(a).to(dt).cuda() for a in (si.q, si.k, si.v))
             beta, gate = torch.from_numpy(si.beta).cuda(), torch.from_numpy(si.gate).cuda()
             keep.append((q, k, v, beta, gate))
+            side = sides[l % 2]
+            main.wait_stream(torch.cuda.current_stream())   # the inputs' copies
             if s % 2 == 0:
                 S.stepq_decode_step(pair.gpu, pools[l], slots, q, k, v, beta, gate, ys[l], wss[l], main, side)
             else:
@@ -67,11 +72,13 @@ def test_overlapped_layers_match_oracle():
                 ev.record(main)
                 side.wait_event(ev)
                 S.stepq_decode_fitpack(pair.gpu, pools[l], slots, k, gate, wss[l], side)
-            y_snap = ys[l].clone()                  # on main, after this layer's readout
+            with torch.cuda.stream(main):
+                y_snap = ys[l].clone()              # on main, after this layer's readout
             with torch.cuda.stream(side):
-                p_snap = pools[l].buf.clone()       # on side, after this layer's fit
+                p_snap = pools[l].buf.clone()       # on the side stream, after this layer's fit
             snaps.append((s, l, si, y_snap, p_snap))
-    main.wait_stream(side)
+    for side in sides:
+        main.wait_stream(side)
     torch.cuda.synchronize()
     worst = 0.0
     for s, l, si, y_snap, p_snap in snaps:
