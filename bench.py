@@ -320,7 +320,11 @@ class DeviceWorkload:
         self.head_bytes = [S.stepq_plan_head_layout(self.plan, h)[1] for h in range(H)]
         self.nslots = cfg.pool_slots
         pool_bytes = self.nslots * self.slot_bytes
-        self.layers = max(1, math.ceil(2 * L2_BYTES / pool_bytes))
+        # at least two layers, as in any model: consecutive calls go to
+        # different layers' pools, so one layer's fit can overlap the next
+        # layer's readout; more when needed to make the cycled pools larger
+        # than twice the L2
+        self.layers = max(2, math.ceil(2 * L2_BYTES / pool_bytes))
         self.slots_np = W.slot_indices(cfg)
         self.slots = torch.from_numpy(self.slots_np).cuda()
         # pack S0 into layer 0, chunk by chunk, then copy into the other layers
