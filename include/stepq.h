@@ -136,7 +136,9 @@ STEPQ_API int stepq_plan_head_layout(const stepq_plan *plan, int32_t head, size_
  * summary, "Method", last paragraph).
  *   dev_buf    device, >= num_slots * slot_bytes bytes, 256-byte aligned.
  * The library allocates a 4-byte device status word and two CUDA events for
- * the pool; stepq_pool_free releases those, never dev_buf.
+ * the pool (and, on the first stepq_decode_step_host call on it, two streams
+ * and three events for that entry's copies); stepq_pool_free releases those,
+ * never dev_buf.
  * Errors: STEPQ_ERR_INVALID (NULL, too small, misaligned), STEPQ_ERR_CUDA.
  */
 STEPQ_API int stepq_pool_alloc(const stepq_plan *plan, int64_t num_slots, void *dev_buf,
@@ -235,9 +237,16 @@ STEPQ_API int stepq_decode_step(const stepq_plan *plan, stepq_pool *pool,
  * The same whole step for callers whose per-token inputs live in host memory
  * (a C caller without a device allocator of its own for them): the call
  * copies q, k, v, beta and gate host -> device into `workspace`, runs
- * stepq_decode_step, and copies y device -> host, all in stream order on
- * main_stream.  Host buffers should be pinned (cudaHostAlloc) for the copies
- * to be asynchronous; y_host is valid once main_stream reaches that point.
+ * stepq_decode_step, and copies y device -> host.  The copies run on two
+ * streams the pool creates on the first such call (and destroys with the
+ * pool): the input copies wait only for this pool's previous fit, not for
+ * earlier work on main_stream, so they overlap the work of the layers before
+ * this one; main_stream waits for them before the readout, and for the copy
+ * of y after it.  So the host inputs may be reused, and y_host is valid, once
+ * main_stream has reached the end of the call's work; the workspace is the
+ * pool's staging area until the call's fit has finished (one workspace per
+ * layer in flight, as for stepq_decode_step).  Host buffers should be pinned
+ * (cudaHostAlloc) for the copies to be asynchronous.
  *   q_host..gate_host, y_host: host, same shapes and types as for
  *             stepq_decode_step.
  *   workspace device, >= stepq_host_workspace_bytes(plan, n, qkv_dtype).

@@ -39,6 +39,9 @@ struct stepq_pool {
     bool fit_pending = false;
     uint32_t test_faults = 0;
     uint64_t wait_limit_ns = stepq::kDefaultWaitLimitNs;
+    // the host-buffer entry's copy streams and events, created on its first call
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
+    cudaEvent_t in_done = nullptr, y_ready = nullptr, y_done = nullptr;
 };
 
 namespace {
@@ -105,6 +108,19 @@ stepq::StepArgs base_args(const stepq_plan *plan, stepq_pool *pool, const int32_
     a.wait_limit_ns = pool->wait_limit_ns;
     (void)plan;
     return a;
+}
+
+// The host-buffer entry's two copy streams and three events, created once
+// per pool on the pool's device.
+int host_streams(stepq_pool *pool) {
+    if (pool->y_done) return STEPQ_OK;
+    cudaError_t e = cudaSuccess;
+    if (!pool->copy_in) e = cudaStreamCreateWithFlags(&pool->copy_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !pool->copy_out) e = cudaStreamCreateWithFlags(&pool->copy_out, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !pool->in_done) e = cudaEventCreateWithFlags(&pool->in_done, cudaEventDisableTiming);
+    if (e == cudaSuccess && !pool->y_ready) e = cudaEventCreateWithFlags(&pool->y_ready, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&pool->y_done, cudaEventDisableTiming);
+    return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "copy streams");
 }
 
 // Make `stream` wait for a fit still pending on the pool's slots.
@@ -332,6 +348,11 @@ int stepq_pool_free(stepq_pool *pool) {
     if (pool->status) cudaFree(pool->status);
     if (pool->readout_done) cudaEventDestroy(pool->readout_done);
     if (pool->fit_done) cudaEventDestroy(pool->fit_done);
+    if (pool->copy_in) cudaStreamDestroy(pool->copy_in);
+    if (pool->copy_out) cudaStreamDestroy(pool->copy_out);
+    if (pool->in_done) cudaEventDestroy(pool->in_done);
+    if (pool->y_ready) cudaEventDestroy(pool->y_ready);
+    if (pool->y_done) cudaEventDestroy(pool->y_done);
     delete pool;
     return STEPQ_OK;
 }
@@ -579,22 +600,36 @@ int stepq_decode_step_host(const stepq_plan *plan, stepq_pool *pool, const int32
         return fail(STEPQ_ERR_INVALID, "workspace of %zu bytes, %zu needed", ws_bytes, L.total);
     uint8_t *w = static_cast<uint8_t *>(workspace);
     cudaStream_t m = static_cast<cudaStream_t>(main_stream);
-    // the staging area must not be overwritten while the previous step's fit
-    // (which reads k and gate from it) is still running
-    if ((rc = wait_pending_fit(pool, m))) return rc;
-    cudaError_t e = cudaMemcpyAsync(w + L.q, q_host, L.qkv_bytes, cudaMemcpyHostToDevice, m);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.k, k_host, L.qkv_bytes, cudaMemcpyHostToDevice, m);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.v, v_host, L.qkv_bytes, cudaMemcpyHostToDevice, m);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.beta, beta_host, L.beta_bytes, cudaMemcpyHostToDevice, m);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.gate, gate_host, L.gate_bytes, cudaMemcpyHostToDevice, m);
+    if ((rc = host_streams(pool))) return rc;
+    // The inputs' copies run on the pool's copy-in stream.  They wait for
+    // this pool's previous fit (which reads k and gate from the staging area,
+    // after its readout read q, k and v), not for earlier work on main_stream,
+    // so they overlap the readouts and copies of the layers before this one.
+    if ((rc = wait_pending_fit(pool, pool->copy_in))) return rc;
+    cudaStream_t ci = pool->copy_in, co = pool->copy_out;
+    cudaError_t e = cudaMemcpyAsync(w + L.q, q_host, L.qkv_bytes, cudaMemcpyHostToDevice, ci);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.k, k_host, L.qkv_bytes, cudaMemcpyHostToDevice, ci);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.v, v_host, L.qkv_bytes, cudaMemcpyHostToDevice, ci);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.beta, beta_host, L.beta_bytes, cudaMemcpyHostToDevice, ci);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.gate, gate_host, L.gate_bytes, cudaMemcpyHostToDevice, ci);
     if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    e = cudaEventRecord(pool->in_done, ci);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(m, pool->in_done, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "copy-in event");
     rc = stepq_decode_step(plan, pool, slot_idx, n, qkv_dtype, w + L.q, w + L.k, w + L.v,
                            reinterpret_cast<const float *>(w + L.beta),
                            reinterpret_cast<const float *>(w + L.gate),
                            reinterpret_cast<float *>(w + L.y), w + L.delta, L.q, main_stream,
                            side_stream);
     if (rc) return rc;
-    e = cudaMemcpyAsync(y_host, w + L.y, L.y_bytes, cudaMemcpyDeviceToHost, m);
+    // y goes back on the copy-out stream; main_stream then waits for it, so
+    // y_host is valid once main_stream has reached this point and the next
+    // readout on main_stream cannot overwrite the staged y before it is read
+    e = cudaEventRecord(pool->y_ready, m);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(co, pool->y_ready, 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(y_host, w + L.y, L.y_bytes, cudaMemcpyDeviceToHost, co);
+    if (e == cudaSuccess) e = cudaEventRecord(pool->y_done, co);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(m, pool->y_done, 0);
     return e == cudaSuccess ? STEPQ_OK : cuda_fail(e, "device-to-host copy");
 }
 
