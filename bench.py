@@ -143,7 +143,8 @@ def parse():
     ap.add_argument("--impl", choices=["stepq", "reference"], default="stepq")
     ap.add_argument("--config", choices=W.CONFIG_ORDER, default="gdn")
     ap.add_argument("--mode", choices=list(MODES), default="stepquant")
-    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--e2e-steps", type=int, default=0,
+                    help="steps of the end-to-end pass (0: as many as the headline's --steps)")
     ap.add_argument("--fp32-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
@@ -1248,7 +1249,9 @@ def main():
     if args.serial and dist.world == 1:
         sm = time_serial(wl, min(args.steps, 5000), args.warmup)
         serial = {"ms_per_step": sm / min(args.steps, 5000)}
-    e2e_ms, h2d, d2h = time_e2e(wl, args.e2e_steps, max(3, args.warmup // 5))
+    if args.e2e_steps <= 0:
+        args.e2e_steps = args.steps
+    e2e_ms, h2d, d2h = time_e2e(wl, args.e2e_steps, args.warmup)
     e2e_ms = dist.max(e2e_ms)
     e2e_value = hu / (e2e_ms / args.e2e_steps * 1e-3)
     graph = time_graph(wl, args.steps) if args.graph else None
@@ -1299,6 +1302,7 @@ def main():
                 "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps,
+                        "steps": args.e2e_steps, "warmup": args.warmup,
                         "path": "stepq_decode_step_host (pinned host q,k,v,beta,gate in, y out)"},
                 "gpu_launches": 2 * args.steps,
                 "clocks": clocks}
