@@ -7,9 +7,11 @@ of the pool's own that the main stream then waits for (the readout emits y
 before the state is requantised: rcap.io post, decode-step pseudocode; the fit
 runs on a separate stream: hyper.ai summary, Method, last paragraph).  This
 test runs it the way a model would: three layers of the full gdn workload (64
-requests x 32 heads), each with its own pool, staging workspace and side
-stream, a high-priority main stream, six steps, fresh pinned inputs and a
-pinned y buffer for every call and nothing synchronised between calls.  The
+requests x 32 heads, six steps) and two layers of the full kda workload (256
+requests x 32 heads with per-row gates and widths, which the step takes in
+chunks of requests; three steps), each layer with its own pool, staging
+workspace and side stream, a high-priority main stream, fresh pinned inputs
+and a pinned y buffer for every call and nothing synchronised between calls.  The
 staging areas are reused every step, so a copy that overtook the previous
 fit of its pool, or a y read back before its readout, would show: after
 every step of every layer, sampled (request, head) blobs of a copy of the
@@ -25,12 +27,14 @@ from gpu_harness import Pair, dev, lib, rel_l2
 
 pytestmark = pytest.mark.gpu
 
-LAYERS, STEPS, SAMPLES = 3, 6, 8
+SAMPLES = 8
 
 
-def test_host_step_layers_match_oracle():
+@pytest.mark.parametrize("name,layers,steps", [("gdn", 3, 6), ("kda", 2, 3)])
+def test_host_step_layers_match_oracle(name, layers, steps):
     import torch
-    cfg = W.CONFIGS["gdn"]
+    cfg = W.CONFIGS[name]
+    LAYERS, STEPS = layers, steps
     pair = Pair(cfg)
     S = lib()
     R, H, d = cfg.requests, cfg.heads, cfg.d
