@@ -135,10 +135,9 @@ STEPQ_API int stepq_plan_head_layout(const stepq_plan *plan, int32_t head, size_
  * per concurrent request ("integrated into the recurrent state pool", hyper.ai
  * summary, "Method", last paragraph).
  *   dev_buf    device, >= num_slots * slot_bytes bytes, 256-byte aligned.
- * The library allocates a 4-byte device status word and two CUDA events for
- * the pool (and, on the first stepq_decode_step_host call on it, two streams
- * and three events for that entry's copies); stepq_pool_free releases those,
- * never dev_buf.
+ * The library allocates a 4-byte device status word, five CUDA events and two
+ * CUDA streams (the copies of stepq_decode_step_host) for the pool;
+ * stepq_pool_free releases those, never dev_buf.
  * Errors: STEPQ_ERR_INVALID (NULL, too small, misaligned), STEPQ_ERR_CUDA.
  */
 STEPQ_API int stepq_pool_alloc(const stepq_plan *plan, int64_t num_slots, void *dev_buf,
@@ -238,8 +237,8 @@ STEPQ_API int stepq_decode_step(const stepq_plan *plan, stepq_pool *pool,
  * (a C caller without a device allocator of its own for them): the call
  * copies q, k, v, beta and gate host -> device into `workspace`, runs
  * stepq_decode_step, and copies y device -> host.  The copies run on two
- * streams the pool creates on the first such call (and destroys with the
- * pool): the input copies wait only for this pool's previous fit, not for
+ * streams the pool owns (created and destroyed with it): the input copies
+ * wait only for this pool's previous fit, not for
  * earlier work on main_stream, so they overlap the work of the layers before
  * this one; main_stream waits for them before the readout, and for the copy
  * of y after it.  So the host inputs may be reused, and y_host is valid, once

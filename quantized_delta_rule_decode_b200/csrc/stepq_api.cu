@@ -110,8 +110,8 @@ stepq::StepArgs base_args(const stepq_plan *plan, stepq_pool *pool, const int32_
     return a;
 }
 
-// The host-buffer entry's two copy streams and three events, created once
-// per pool on the pool's device.
+// The host-buffer entry's two copy streams and three events, created with
+// the pool on its device (the entry checks again, in case creation failed).
 int host_streams(stepq_pool *pool) {
     if (pool->y_done) return STEPQ_OK;
     cudaError_t e = cudaSuccess;
@@ -337,6 +337,15 @@ int stepq_pool_alloc(const stepq_plan *plan, int64_t num_slots, void *dev_buf, s
         if (p->readout_done) cudaEventDestroy(p->readout_done);
         delete p;
         return cuda_fail(e, "pool status/events");
+    }
+    // the host-buffer entry's copy streams, made here so that no call of it
+    // pays for their creation
+    int rc2 = host_streams(p);
+    if (rc2) {
+        const std::string msg = g_err;   // stepq_pool_free clears the message
+        stepq_pool_free(p);
+        g_err = msg;
+        return rc2;
     }
     *out = p;
     return STEPQ_OK;
